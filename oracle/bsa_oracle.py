@@ -1,0 +1,427 @@
+"""CPU oracle for block-sparse causal attention: plain, slow, fp64.
+
+TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+benchmark's CPU-baseline leg may import or run this module. The product path
+(the CUDA library and its binding) never calls it, and it imports nothing
+from the product.
+
+Sources (summary pages, cited by title and section):
+
+* [UGS] "Resumo Técnico: Seleção com Portão de Incerteza para Atenção de
+  Esparsidade em Blocos" -- Metodologia steps 1-5 (block scoring backbone,
+  per-tile top-k with the tile's max over rows, the normalised cut margin
+  sigma, head mean + per-layer quantile trigger, rho*k expansion with
+  sentinel-padded kv_idx).
+* [Stem] "Stem: Rethinking Causal Information Flow in Sparse Attention" --
+  Resumo técnico, 2. Metodologia, A (Token Position-Decay budget), B
+  (Output-Aware Metric) and "Implementação" (block downsampling, dynamic
+  budget, sparse aggregation).
+* [ART] "Resumo Técnico: ART (Attention Run-time Termination)" -- 2.1
+  (tile-wise streaming exposes the partial output O^(t)), 2.2 (probe vector,
+  d_scale and d_direction against tau and phi), 2.3 (patience p), 2.4
+  (block 0 always evaluated).
+
+Conventions: inputs are bf16 values widened exactly to fp64 (or fp32 values
+widened); arithmetic is fp64 unless a step says fp32. Layouts: Q [B,Hq,N,d],
+K and V [B,Hkv,N,d]; query head h reads KV head h // (Hq // Hkv).
+
+Readings taken where the pages are silent (each is also listed in the design
+notes): no 1/sqrt(d) factor in block scores; the tile max runs over all rows
+of the tile, unmasked; the blocks that intersect the tile's own rows are
+always kept and count toward k; ties in the ranking go to the lower block
+index; sigma of a non-cut tile is 1; the quantile is the linear-interpolation
+empirical quantile over the cut tiles of the call; the trigger compares
+strictly (sigma_bar < theta) and is shared by all heads of a (batch, tile);
+the sentinel is -1. For decode: the probe is a fixed set of coordinates of the
+first query head of the KV group; d_scale is the absolute difference of the
+probe norms; d_direction is 1 - cosine, taken as 1 when a norm is zero;
+termination is decided per (batch, KV head).
+
+Parity status: every function below is pinned by CPU tests against closed
+forms, library routines (torch scaled_dot_product_attention, numpy.quantile)
+or brute force -- except the exact termination block on random decode data,
+which the pages do not fix ("parity unpinned" for that value; the decision
+rule itself is pinned by hand-worked traces).
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+NEG_INF32 = np.float32(-np.inf)
+
+
+def widen(x: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) or float32 values -> float64, exactly."""
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# tile geometry and budget
+
+def tile_blocks(t: int, tile_q: int, block_k: int):
+    """Key blocks touched by query tile t.
+
+    Returns (f_lo, J): the forced blocks are f_lo..J (the blocks that
+    intersect the tile's own rows, J = the block of the tile's last row) and
+    the scored candidates are 0..f_lo-1. [UGS step 2] selects per query tile;
+    keeping the diagonal block is the causal self-visibility rule.
+    """
+    f_lo = (t * tile_q) // block_k
+    J = ((t + 1) * tile_q - 1) // block_k
+    return f_lo, J
+
+
+def budget_k(t: int, n_qt: int, k_first: int, k_last: int) -> int:
+    """Per-tile budget k_t. [Stem, 2.A, TPD]: linear decay from the first to the
+    last tile, k_t = k_first - floor((k_first - k_last) * t / (n_qt - 1));
+    with k_first == k_last this is the fixed top-k of [UGS step 2]."""
+    if n_qt <= 1 or k_first == k_last:
+        return k_first
+    return k_first - ((k_first - k_last) * t) // (n_qt - 1)
+
+
+def tile_slots(t: int, n_qt: int, tile_q: int, block_k: int,
+               k_first: int, k_last: int, rho: int):
+    """(n_forced, n_cand, m_t, M_t): forced block count, candidate count,
+    scored slots at the base budget and at the rho-expanded budget
+    [UGS step 5: top-rho*k instead of top-k], both capped at the J_t+1 blocks
+    the tile can see and never below the forced blocks."""
+    f_lo, J = tile_blocks(t, tile_q, block_k)
+    nF = J - f_lo + 1
+    k = budget_k(t, n_qt, k_first, k_last)
+    K = max(nF, min(k, J + 1))
+    KM = max(nF, min(rho * k, J + 1))
+    return nF, f_lo, K - nF, KM - nF
+
+
+def kv_idx_width(N: int, tile_q: int, block_k: int, k_first: int, k_last: int, rho: int) -> int:
+    """Uniform kv_idx row width W (data independent), [UGS step 5 uniform dispatch shape]."""
+    n_kb = N // block_k
+    f_max = max(1, tile_q // block_k)      # most forced blocks any tile has
+    return min(n_kb, max(rho * max(k_first, k_last), f_max))
+
+
+# ---------------------------------------------------------------------------
+# a1/a2: pooling and block scores
+
+def pool_keys(K: np.ndarray, block_k: int) -> np.ndarray:
+    """K_bar[..., j, :] = mean of the block_k keys of block j ([UGS step 1],
+    mean-pooled keys; [Stem, Implementação] block downsampling). fp64."""
+    K = widen(K)
+    *lead, N, d = K.shape
+    return K.reshape(*lead, N // block_k, block_k, d).mean(axis=-2)
+
+
+def value_block_norm(V: np.ndarray, block_k: int) -> np.ndarray:
+    """w[..., j] = || mean of the block's V rows ||_2 (output-aware block weight,
+    motivated by [Stem, 2.B]: value magnitude enters the metric). fp64."""
+    Vb = pool_keys(V, block_k)
+    return np.sqrt((Vb * Vb).sum(axis=-1))
+
+
+def score_tile(Q_tile: np.ndarray, Kbar: np.ndarray, J: int,
+               w: Optional[np.ndarray] = None) -> np.ndarray:
+    """One row of block scores for a query tile ([UGS step 2]: the tile's block
+    score is the max over the tile's rows of q_i . K_bar_j).
+
+    Q_tile [tile_q, d], Kbar [n_kb, d] (fp64). Blocks j > J are not visible
+    to any row of the tile and score -inf. With w given (output-aware form),
+    the max is multiplied by w_j in fp64 before rounding. Returns fp32.
+    """
+    Q_tile = widen(Q_tile)
+    n_kb = Kbar.shape[0]
+    out = np.full(n_kb, NEG_INF32, dtype=np.float32)
+    dots = Q_tile @ Kbar[: J + 1].T            # [tile_q, J+1]
+    s = dots.max(axis=0)
+    if w is not None:
+        s = s * w[: J + 1]
+    out[: J + 1] = s.astype(np.float32)
+    return out
+
+
+def block_scores(Q: np.ndarray, K: np.ndarray, tile_q: int, block_k: int,
+                 V: Optional[np.ndarray] = None, Hkv: Optional[int] = None) -> np.ndarray:
+    """scores [B, Hq, n_qt, n_kb] fp32; V given -> output-aware form."""
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    n_qt, n_kb = N // tile_q, N // block_k
+    out = np.empty((B, Hq, n_qt, n_kb), np.float32)
+    for b in range(B):
+        for g in range(Hkv):
+            Kbar = pool_keys(K[b, g], block_k)
+            w = value_block_norm(V[b, g], block_k) if V is not None else None
+            for h in range(g * G, (g + 1) * G):
+                Qh = widen(Q[b, h])
+                for t in range(n_qt):
+                    _, J = tile_blocks(t, tile_q, block_k)
+                    out[b, h, t] = score_tile(Qh[t * tile_q:(t + 1) * tile_q], Kbar, J, w)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# a4: ranking and the cut margin sigma
+
+def rank_candidates(s_row: np.ndarray, n_cand: int) -> np.ndarray:
+    """Candidate blocks 0..n_cand-1 ordered by (score descending, index
+    ascending). Raises on a non-finite candidate score."""
+    s = np.asarray(s_row[:n_cand], dtype=np.float32)
+    if not np.all(np.isfinite(s)):
+        raise ValueError("non-finite candidate score")
+    idx = np.arange(n_cand)
+    return np.lexsort((idx, -s)).astype(np.int64)
+
+
+def cut_margin(s_row: np.ndarray, order: np.ndarray, m: int) -> np.float32:
+    """sigma = (s_(m-1) - s_(m)) / (s_(0) - s_(m)) in fp32 ([UGS step 3]), with
+    ranks 0-based over the ordered candidates; an all-tied head (0/0) gives 0."""
+    s = np.asarray(s_row, dtype=np.float32)
+    top, km1, km = s[order[0]], s[order[m - 1]], s[order[m]]
+    num = np.float32(km1 - km)
+    den = np.float32(top - km)
+    if den == 0:
+        return np.float32(0.0)
+    return np.float32(num / den)
+
+
+def select(scores: np.ndarray, tile_q: int, block_k: int, k_first: int, k_last: int,
+           rho: int, gate_quantile: float, gate_threshold: float = float("nan")):
+    """a3-a6: budget, ranking, sigma, gate and kv_idx for a whole layer call.
+
+    scores [B, Hq, n_qt, n_kb] fp32. Returns a dict with kv_idx [B,Hq,n_qt,W]
+    (ascending, -1 padded), kv_cnt, sigma [B,Hq,n_qt], sigma_bar [B,n_qt],
+    trigger [B,n_qt] (uint8), theta (fp32 scalar, NaN when undefined), cut
+    [n_qt] (bool) and W.
+    """
+    B, Hq, n_qt, n_kb = scores.shape
+    N = n_kb * block_k
+    W = kv_idx_width(N, tile_q, block_k, k_first, k_last, rho)
+    sigma = np.ones((B, Hq, n_qt), np.float32)
+    cut = np.zeros(n_qt, bool)
+    ranked = {}
+    slots = [tile_slots(t, n_qt, tile_q, block_k, k_first, k_last, rho) for t in range(n_qt)]
+    for t in range(n_qt):
+        nF, n_cand, m, M = slots[t]
+        cut[t] = n_cand > m >= 1
+        for b in range(B):
+            for h in range(Hq):
+                order = rank_candidates(scores[b, h, t], n_cand)
+                ranked[b, h, t] = order
+                if cut[t]:
+                    sigma[b, h, t] = cut_margin(scores[b, h, t], order, m)
+
+    sigma_bar, theta, trigger = gate(sigma, cut, rho, gate_quantile, gate_threshold)
+
+    kv_idx = np.full((B, Hq, n_qt, W), -1, np.int32)
+    kv_cnt = np.zeros((B, Hq, n_qt), np.int32)
+    for t in range(n_qt):
+        nF, n_cand, m, M = slots[t]
+        forced = np.arange(n_cand, n_cand + nF)
+        for b in range(B):
+            take = M if trigger[b, t] else m
+            for h in range(Hq):
+                sel = np.sort(np.concatenate([ranked[b, h, t][:take], forced]))
+                kv_idx[b, h, t, : len(sel)] = sel
+                kv_cnt[b, h, t] = len(sel)
+    return dict(kv_idx=kv_idx, kv_cnt=kv_cnt, sigma=sigma, sigma_bar=sigma_bar,
+                trigger=trigger, theta=theta, cut=cut, W=W)
+
+
+# ---------------------------------------------------------------------------
+# a5: gate
+
+def head_mean(sigma: np.ndarray) -> np.ndarray:
+    """sigma_bar[b, t] = (sum over heads in order h = 0..Hq-1, fp32) / Hq in fp32
+    ([UGS step 4]: per-head sigma averaged into one signal per query tile)."""
+    B, Hq, n_qt = sigma.shape
+    acc = np.zeros((B, n_qt), np.float32)
+    for h in range(Hq):
+        acc = (acc + sigma[:, h, :]).astype(np.float32)
+    return (acc / np.float32(Hq)).astype(np.float32)
+
+
+def empirical_quantile(values: np.ndarray, q: float) -> np.float32:
+    """Linear-interpolation empirical quantile with a fixed operation order:
+    pos = q*(M-1) (fp64), lo = floor(pos), hi = min(lo+1, M-1),
+    f = fp32(pos - lo), theta = v_lo + f*(v_hi - v_lo) with fp32 rounding
+    after each operation. NaN for an empty population."""
+    v = np.sort(np.asarray(values, dtype=np.float32))
+    M = len(v)
+    if M == 0:
+        return np.float32(np.nan)
+    pos = float(np.float32(q)) * (M - 1)
+    lo = int(math.floor(pos))
+    hi = min(lo + 1, M - 1)
+    f = np.float32(pos - lo)
+    diff = np.float32(v[hi] - v[lo])
+    return np.float32(v[lo] + np.float32(f * diff))
+
+
+def gate(sigma: np.ndarray, cut: np.ndarray, rho: int, q: float,
+         fixed_threshold: float = float("nan")):
+    """Head mean, per-layer quantile threshold theta over the cut tiles of the
+    call, and trigger = cut and sigma_bar < theta ([UGS step 4]). With rho == 1
+    nothing expands, so no trigger is raised and theta is NaN. A negative q
+    selects a fixed, externally calibrated threshold instead."""
+    sigma_bar = head_mean(sigma)
+    B, n_qt = sigma_bar.shape
+    trigger = np.zeros((B, n_qt), np.uint8)
+    if rho <= 1:
+        return sigma_bar, np.float32(np.nan), trigger
+    if q < 0:
+        theta = np.float32(fixed_threshold)
+    else:
+        theta = empirical_quantile(sigma_bar[:, cut].reshape(-1), q)
+    trig = (sigma_bar < theta) & cut[None, :]
+    return sigma_bar, theta, trig.astype(np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# a7: block-sparse attend
+
+def attend_tile(Q_tile: np.ndarray, K: np.ndarray, V: np.ndarray, kv_row: np.ndarray,
+                row0: int, block_k: int, scale: float):
+    """Softmax attention of the tile's rows over the listed key blocks
+    ([UGS step 5], [Stem, Implementação]: sparse aggregation over the selected
+    blocks), with the causal rule key <= query. K, V [N, d] of the head's KV
+    group. Returns (O [rows, d], lse [rows]) in fp64; lse is the natural log of
+    the softmax denominator."""
+    Qt = widen(Q_tile)
+    blocks = [int(j) for j in kv_row if j >= 0]
+    keys = np.concatenate([np.arange(j * block_k, (j + 1) * block_k) for j in blocks])
+    Kt, Vt = widen(K[keys]), widen(V[keys])
+    logits = scale * (Qt @ Kt.T)
+    rows = row0 + np.arange(Qt.shape[0])
+    logits[keys[None, :] > rows[:, None]] = -np.inf
+    mx = logits.max(axis=1, keepdims=True)
+    p = np.exp(logits - mx)
+    den = p.sum(axis=1, keepdims=True)
+    return (p @ Vt) / den, (mx + np.log(den))[:, 0]
+
+
+def attend(Q, K, V, kv_idx, tile_q, block_k, scale, tiles=None):
+    """O [B,Hq,N,d] fp64 and lse [B,Hq,N]; with ``tiles`` (a list of (b, h, t))
+    only those tiles are computed and the rest is left NaN."""
+    B, Hq, N, d = Q.shape
+    G = Hq // K.shape[1]
+    O = np.full((B, Hq, N, d), np.nan)
+    lse = np.full((B, Hq, N), np.nan)
+    if tiles is None:
+        tiles = [(b, h, t) for b in range(B) for h in range(Hq) for t in range(N // tile_q)]
+    for b, h, t in tiles:
+        r0 = t * tile_q
+        o, l = attend_tile(Q[b, h, r0:r0 + tile_q], K[b, h // G], V[b, h // G],
+                           kv_idx[b, h, t], r0, block_k, scale)
+        O[b, h, r0:r0 + tile_q] = o
+        lse[b, h, r0:r0 + tile_q] = l
+    return O, lse
+
+
+def dense_causal_attention(Q, K, V, scale):
+    """Textbook softmax(scale * Q K^T + causal mask) V for [N, d] operands, fp64."""
+    Q, K, V = widen(Q), widen(K), widen(V)
+    N = Q.shape[0]
+    logits = scale * (Q @ K.T)
+    logits[np.triu(np.ones((N, N), bool), 1)] = -np.inf
+    p = np.exp(logits - logits.max(axis=1, keepdims=True))
+    return (p / p.sum(axis=1, keepdims=True)) @ V
+
+
+# ---------------------------------------------------------------------------
+# a8: decode with run-time termination
+
+def probe_step(x_prev: Sequence[float], x_cur: Sequence[float]):
+    """(d_scale, d_direction) between consecutive probes ([ART, 2.2]):
+    the absolute difference of their L2 norms and one minus their cosine.
+    fp64 on the fp32 probe values; every sum runs in index order with a
+    separate multiply and add; d_direction = 1 when a norm is zero."""
+    s_cur = 0.0
+    s_prev = 0.0
+    dot = 0.0
+    for a, b in zip(x_cur, x_prev):
+        a = float(a)
+        b = float(b)
+        s_cur = s_cur + a * a
+        s_prev = s_prev + b * b
+        dot = dot + a * b
+    n_cur = math.sqrt(s_cur)
+    n_prev = math.sqrt(s_prev)
+    d_scale = abs(n_cur - n_prev)
+    den = n_cur * n_prev
+    d_dir = 1.0 if den == 0.0 else 1.0 - dot / den
+    return d_scale, d_dir
+
+
+def termination_block(trace: np.ndarray, tau: float, phi: float, patience: int,
+                      n_blocks: Optional[int] = None) -> int:
+    """blocks_used from a probe trace [n_blocks, n_probe] (fp32): block 0 is
+    always processed ([ART, 2.4]); after each block t >= 1 the block is stable
+    iff d_scale < tau and d_direction < phi ([ART, 2.2]); streaming stops after
+    block t once ``patience`` consecutive stable blocks end at t ([ART, 2.3]).
+    Returns t+1, or the total block count when it never stops. tau and phi are
+    compared as fp32 parameters widened to fp64."""
+    trace = np.asarray(trace, dtype=np.float32)
+    n = trace.shape[0] if n_blocks is None else n_blocks
+    tau64 = float(np.float32(tau))
+    phi64 = float(np.float32(phi))
+    run = 0
+    for t in range(1, n):
+        ds, dd = probe_step(trace[t - 1], trace[t])
+        if ds < tau64 and dd < phi64:
+            run += 1
+        else:
+            run = 0
+        if run >= patience:
+            return t + 1
+    return n
+
+
+def decode_group(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, block_kv: int, scale: float,
+                 tau: float, phi: float, patience: int, probe_dims: np.ndarray,
+                 enable: bool = True):
+    """One (batch, KV head): q [G, d] (the group's query heads), caches [L, d].
+
+    Blocks 0, 1, ... of block_kv keys are visited in order ([ART, 2.1]); after
+    block t the normalised partial output O^(t) of each head is the softmax
+    over all keys of blocks 0..t applied to V (fp64; the common max shift
+    cancels in the ratio). The probe x^(t) is O^(t) of the group's first head
+    at ``probe_dims``, rounded to fp32. Returns (O [G, d] fp64 at the final
+    block, blocks_used, trace [n_blocks, n_probe] fp32 up to blocks_used).
+    """
+    qf, Kf, Vf = widen(q), widen(Kc), widen(Vc)
+    L = Kf.shape[0]
+    nb = L // block_kv
+    logits = scale * (qf @ Kf.T)                       # [G, L]
+    mx = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - mx)
+    eb = e.reshape(e.shape[0], nb, block_kv)
+    num = np.cumsum(np.einsum("gbk,bkd->gbd", eb, Vf.reshape(nb, block_kv, -1)), axis=1)
+    den = np.cumsum(eb.sum(axis=2), axis=1)            # [G, nb]
+    partial = num / den[:, :, None]                    # O^(t) for every t: [G, nb, d]
+    trace = partial[0][:, probe_dims].astype(np.float32)
+    used = termination_block(trace, tau, phi, patience) if enable else nb
+    return partial[:, used - 1, :], used, trace[:used]
+
+
+def decode(q, Kc, Vc, block_kv, scale, tau, phi, patience, probe_dims, enable=True):
+    """q [B,Hq,d], caches [B,Hkv,L,d] -> (O [B,Hq,d] fp64, blocks_used [B,Hkv],
+    traces dict {(b, g): trace})."""
+    B, Hq, d = q.shape
+    Hkv = Kc.shape[1]
+    G = Hq // Hkv
+    O = np.empty((B, Hq, d))
+    used = np.empty((B, Hkv), np.int32)
+    traces = {}
+    for b in range(B):
+        for g in range(Hkv):
+            o, u, tr = decode_group(q[b, g * G:(g + 1) * G], Kc[b, g], Vc[b, g], block_kv,
+                                    scale, tau, phi, patience, probe_dims, enable)
+            O[b, g * G:(g + 1) * G] = o
+            used[b, g] = u
+            traces[b, g] = tr
+    return O, used, traces

@@ -1,0 +1,473 @@
+"""Pins for the CPU oracle: it is checked against things other than itself
+(hand-worked fixtures, closed forms, library routines, brute force).
+
+Sources: "Resumo Técnico: Seleção com Portão de Incerteza para Atenção de
+Esparsidade em Blocos" (Metodologia steps 1-5), "Stem: Rethinking Causal
+Information Flow in Sparse Attention" (2. Metodologia A and B),
+"Resumo Técnico: ART (Attention Run-time Termination)" (2.1-2.4).
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import bsa_oracle as O
+from block_sparse_causal_bsa_b200 import synthetic as S
+
+
+def _parse_float(s):
+    return float("-inf") if s == "-inf" else float(s)
+
+
+# ---------------------------------------------------------------------------
+# sigma (hand-worked fixture)
+
+def test_cut_margin_golden(golden_dir):
+    n = 0
+    for line in open(os.path.join(golden_dir, "cut_margin.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        m, scores, sigma, _ = [p.strip() for p in line.split(";")]
+        s = np.array([float(x) for x in scores.split()], np.float32)
+        order = O.rank_candidates(s, len(s))
+        got = O.cut_margin(s, order, int(m))
+        assert got == np.float32(float(sigma)), (line, got)
+        n += 1
+    assert n == 8
+
+
+def test_sigma_in_unit_interval_and_ties():
+    rng = np.random.default_rng(0)
+    for _ in range(2000):
+        n = int(rng.integers(2, 40))
+        m = int(rng.integers(1, n))
+        s = rng.standard_normal(n).astype(np.float32) * np.float32(10 ** rng.uniform(-3, 3))
+        order = O.rank_candidates(s, n)
+        sig = O.cut_margin(s, order, m)
+        assert 0.0 <= sig <= 1.0
+        # plant an exact tie across the cut: the block ranked m gets the score of rank m-1
+        s2 = s.copy()
+        s2[order[m]] = s2[order[m - 1]]
+        o2 = O.rank_candidates(s2, n)
+        assert O.cut_margin(s2, o2, m) == 0.0
+    # a dominant kept set with a flat tail: sigma = 1 exactly
+    s = np.array([9, 9, 9, 0, 0, 0], np.float32)
+    assert O.cut_margin(s, O.rank_candidates(s, 6), 3) == 1.0
+
+
+def test_rank_rejects_nonfinite():
+    with pytest.raises(ValueError):
+        O.rank_candidates(np.array([1, np.nan, 0], np.float32), 3)
+    with pytest.raises(ValueError):
+        O.rank_candidates(np.array([1, -np.inf, 0], np.float32), 3)
+
+
+# ---------------------------------------------------------------------------
+# top-k ranking against brute-force subset enumeration
+
+def test_topk_brute_force():
+    """For tiny rows, exactly one subset of size m has every kept block ranked
+    above every dropped block under (score desc, index asc); it must equal the
+    oracle's first m."""
+    rng = np.random.default_rng(1)
+    for _ in range(300):
+        n = int(rng.integers(1, 8))
+        m = int(rng.integers(0, n + 1))
+        s = rng.integers(-3, 4, size=n).astype(np.float32)   # many ties
+        def better(a, b):
+            return s[a] > s[b] or (s[a] == s[b] and a < b)
+        good = []
+        for sub in itertools.combinations(range(n), m):
+            kept = set(sub)
+            if all(better(a, b) for a in kept for b in range(n) if b not in kept):
+                good.append(kept)
+        assert len(good) == 1
+        assert set(O.rank_candidates(s, n)[:m].tolist()) == good[0]
+
+
+# ---------------------------------------------------------------------------
+# budget
+
+def test_tpd_budget_golden(golden_dir):
+    for line in open(os.path.join(golden_dir, "tpd_budget.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        t, k, _ = [p.strip() for p in line.split(";")]
+        assert O.budget_k(int(t), 512, 128, 32) == int(k)
+
+
+def test_budget_properties():
+    for n_qt, kf, kl in [(512, 128, 32), (7, 10, 3), (1, 5, 2), (100, 64, 64)]:
+        ks = [O.budget_k(t, n_qt, kf, kl) for t in range(n_qt)]
+        assert ks[0] == kf and ks[-1] == (kl if n_qt > 1 else kf)
+        assert all(a >= b for a, b in zip(ks, ks[1:]))
+        assert all(kl <= k <= kf for k in ks)
+
+
+def test_slots_and_width():
+    # tile 128, blocks of 64: two forced blocks per tile, candidates 0..2t-1
+    nF, nc, m, M = O.tile_slots(0, 1024, 128, 64, 64, 64, 2)
+    assert (nF, nc, m, M) == (2, 0, 0, 0)
+    nF, nc, m, M = O.tile_slots(10, 1024, 128, 64, 64, 64, 2)
+    assert (nF, nc, m, M) == (2, 20, 20, 20)          # budget above the 22 visible blocks
+    nF, nc, m, M = O.tile_slots(40, 1024, 128, 64, 64, 64, 2)
+    assert (nF, nc, m, M) == (2, 80, 62, 80)
+    nF, nc, m, M = O.tile_slots(500, 1024, 128, 64, 64, 64, 2)
+    assert (nF, nc, m, M) == (2, 1000, 62, 126)
+    assert O.kv_idx_width(131072, 128, 64, 64, 64, 2) == 128
+    assert O.kv_idx_width(1024, 64, 64, 4, 4, 1) == 4
+    assert O.kv_idx_width(65536, 128, 64, 128, 32, 1) == 128
+    # forced blocks exceed a tiny budget
+    nF, nc, m, M = O.tile_slots(5, 16, 128, 64, 1, 1, 1)
+    assert (nF, m) == (2, 0)
+    assert O.kv_idx_width(2048, 128, 64, 1, 1, 1) == 2
+    # key blocks larger than the query tile: one forced block
+    assert O.tile_blocks(5, 64, 128) == (2, 2)
+
+
+# ---------------------------------------------------------------------------
+# select / gate / finalize on the hand-worked layer
+
+def _load_select_tiny(golden_dir):
+    scores, kv, sig, trig, theta = {}, {}, {}, {}, None
+    for line in open(os.path.join(golden_dir, "select_tiny.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        head, rest = line.split(":", 1)
+        head = head.split()
+        if head[0] == "scores":
+            scores[int(head[1])] = [_parse_float(x) for x in rest.split()]
+        elif head[0] == "kv":
+            a, b, c = rest.split(";")
+            kv[int(head[1])] = [int(x) for x in a.split()]
+            sig[int(head[1])] = np.float32(float(b))
+            trig[int(head[1])] = int(c)
+        elif head[0] == "theta":
+            theta = np.float32(float(rest))
+    return scores, kv, sig, trig, theta
+
+
+def test_select_golden(golden_dir):
+    scores, kv, sig, trig, theta = _load_select_tiny(golden_dir)
+    s = np.array([[[scores[t] for t in range(6)]]], np.float32)
+    r = O.select(s, 64, 64, 3, 3, 2, 0.5)
+    assert r["W"] == 6
+    for t in range(6):
+        assert r["kv_idx"][0, 0, t].tolist() == kv[t]
+        assert r["kv_cnt"][0, 0, t] == sum(1 for x in kv[t] if x >= 0)
+        assert r["sigma"][0, 0, t] == sig[t]
+        assert r["trigger"][0, t] == trig[t]
+    assert r["theta"] == theta
+
+
+def test_gate_quantile_matches_numpy():
+    rng = np.random.default_rng(2)
+    for M in [1, 2, 3, 10, 257, 1024]:
+        v = rng.random(M).astype(np.float32)
+        for q in [0.0, 0.1, 0.25, 0.5, 0.9, 1.0]:
+            th = O.empirical_quantile(v, q)
+            ref = np.quantile(v.astype(np.float64), float(np.float32(q)), method="linear")
+            assert abs(float(th) - ref) <= 4 * np.spacing(np.float32(max(abs(ref), 1e-30)))
+
+
+def test_gate_trigger_counts():
+    rng = np.random.default_rng(3)
+    B, Hq, n_qt = 2, 4, 50
+    sigma = rng.random((B, Hq, n_qt)).astype(np.float32)
+    cut = np.ones(n_qt, bool)
+    cut[:5] = False
+    sigma[:, :, :5] = 1.0
+    sbar, theta, trig = O.gate(sigma, cut, 2, 0.25)
+    assert trig.sum() == int(((sbar < theta) & cut[None]).sum())
+    assert trig[:, :5].sum() == 0
+    # about a quarter of the cut tiles fall strictly below the 25% quantile
+    assert abs(trig.sum() - 0.25 * B * 45) <= 2
+    # q = 0: theta = min, strict comparison -> nothing triggers
+    _, th0, t0 = O.gate(sigma, cut, 2, 0.0)
+    assert t0.sum() == 0 and th0 == sbar[:, cut].min()
+    # rho = 1: no expansion, no trigger
+    _, thn, tn = O.gate(sigma, cut, 1, 0.25)
+    assert tn.sum() == 0 and np.isnan(thn)
+    # fixed external threshold
+    _, thf, tf = O.gate(sigma, cut, 2, -1.0, 0.5)
+    assert thf == np.float32(0.5) and tf.sum() == int(((sbar < 0.5) & cut[None]).sum())
+
+
+def test_head_mean_order():
+    # fp32 sum in head order then a correctly rounded divide
+    sigma = np.array([[[1e-8]], [[1.0]], [[-1.0]]], np.float32).reshape(1, 3, 1)
+    sb = O.head_mean(sigma)
+    acc = np.float32(np.float32(np.float32(0) + np.float32(1e-8)) + np.float32(1.0))
+    acc = np.float32(acc + np.float32(-1.0))
+    assert sb[0, 0] == np.float32(acc / np.float32(3))
+
+
+def test_select_structure_random():
+    rng = np.random.default_rng(4)
+    B, Hq, tile_q, bk, N = 2, 3, 128, 64, 64 * 40
+    n_qt, n_kb = N // tile_q, N // bk
+    scores = rng.standard_normal((B, Hq, n_qt, n_kb)).astype(np.float32)
+    for t in range(n_qt):
+        scores[:, :, t, O.tile_blocks(t, tile_q, bk)[1] + 1:] = -np.inf
+    r = O.select(scores, tile_q, bk, 8, 4, 2, 0.3)
+    W = r["W"]
+    assert W == 16
+    for b in range(B):
+        for h in range(Hq):
+            for t in range(n_qt):
+                nF, nc, m, M = O.tile_slots(t, n_qt, tile_q, bk, 8, 4, 2)
+                row = r["kv_idx"][b, h, t]
+                cnt = r["kv_cnt"][b, h, t]
+                assert cnt == nF + (M if r["trigger"][b, t] else m)
+                assert np.all(row[cnt:] == -1) and np.all(row[:cnt] >= 0)
+                assert np.all(np.diff(row[:cnt]) > 0)
+                assert set(range(nc, nc + nF)) <= set(row[:cnt].tolist())
+                # the kept candidates outrank every dropped candidate
+                kept = [j for j in row[:cnt] if j < nc]
+                drop = [j for j in range(nc) if j not in kept]
+                if kept and drop:
+                    s = scores[b, h, t]
+                    assert min(s[kept]) >= max(s[drop])
+
+
+# ---------------------------------------------------------------------------
+# pooling and scores (closed forms)
+
+def test_pool_closed_form():
+    rng = np.random.default_rng(5)
+    bk, d, nb = 64, 16, 5
+    a = rng.standard_normal((nb, d))
+    u = rng.standard_normal((nb, d))
+    offs = np.arange(bk) - (bk - 1) / 2.0          # zero-sum offsets
+    K = (a[:, None, :] + offs[None, :, None] * u[:, None, :] / 64).reshape(nb * bk, d)
+    Kb = O.pool_keys(K.astype(np.float32).astype(np.float64), bk)
+    np.testing.assert_allclose(Kb, a, atol=1e-6)
+    # value-block weight: rows v_j + zero-sum offsets, v_j = c_j * (3, 4, 0, ...)
+    c = rng.random(nb) + 0.5
+    v = np.zeros((nb, d))
+    v[:, 0], v[:, 1] = 3 * c, 4 * c
+    V = (v[:, None, :] + offs[None, :, None] * u[:, None, :] / 64).reshape(nb * bk, d)
+    np.testing.assert_allclose(O.value_block_norm(V, bk), 5 * c, rtol=1e-12)
+
+
+def test_score_closed_forms():
+    rng = np.random.default_rng(6)
+    tile_q, bk, d, N = 4, 2, 8, 16
+    n_kb = N // bk
+    Kb = rng.standard_normal((n_kb, d))
+    # one-hot query rows pick coordinates: score = max of the picked coordinates of K_bar_j
+    cols = np.array([1, 5, 5, 2])
+    Qt = np.zeros((tile_q, d))
+    Qt[np.arange(tile_q), cols] = 1.0
+    J = 5
+    s = O.score_tile(Qt, Kb, J)
+    exp = Kb[:, [1, 5, 2]].max(axis=1).astype(np.float32)
+    assert np.array_equal(s[: J + 1], exp[: J + 1])
+    assert np.all(np.isneginf(s[J + 1:]))
+    # output-aware form multiplies the max by w_j (negative max gets more negative)
+    w = rng.random(n_kb) + 0.1
+    s2 = O.score_tile(Qt, Kb, J, w)
+    assert np.array_equal(s2[: J + 1], (Kb[:, [1, 5, 2]].max(axis=1) * w).astype(np.float32)[: J + 1])
+
+
+def test_score_equals_mean_of_key_dots():
+    """q . K_bar_j = (1/bk) sum_r q . k_r (linearity), checked per key."""
+    rng = np.random.default_rng(7)
+    B, Hq, Hkv, N, d, tile_q, bk = 1, 4, 2, 256, 16, 32, 16
+    Q = rng.standard_normal((B, Hq, N, d)).astype(np.float32)
+    K = rng.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    s = O.block_scores(Q, K, tile_q, bk)
+    n_qt, n_kb = N // tile_q, N // bk
+    finite = 0
+    for h in range(Hq):
+        g = h // 2
+        per_key = Q[0, h].astype(np.float64) @ K[0, g].astype(np.float64).T      # [N, N]
+        for t in range(n_qt):
+            rows = per_key[t * tile_q:(t + 1) * tile_q]
+            for j in range(n_kb):
+                ref = rows[:, j * bk:(j + 1) * bk].mean(axis=1).max()
+                if j <= ((t + 1) * tile_q - 1) // bk:
+                    assert abs(s[0, h, t, j] - ref) <= 1e-6 * max(1.0, abs(ref))
+                    finite += 1
+                else:
+                    assert np.isneginf(s[0, h, t, j])
+    assert finite == Hq * sum(((t + 1) * tile_q - 1) // bk + 1 for t in range(n_qt))
+
+
+# ---------------------------------------------------------------------------
+# attend: full budget reduces to dense causal attention (library routine)
+
+def _sdpa(Q, K, V, scale):
+    q = torch.from_numpy(O.widen(Q))[None, None]
+    k = torch.from_numpy(O.widen(K))[None, None]
+    v = torch.from_numpy(O.widen(V))[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(
+        q, k, v, is_causal=True, scale=scale)[0, 0].numpy()
+
+
+@pytest.mark.parametrize("tile_q,bk", [(64, 64), (128, 64), (64, 128)])
+def test_attend_full_budget_is_dense(tile_q, bk):
+    rng = np.random.default_rng(8)
+    N, d, Hq, Hkv = 512, 32, 4, 2
+    Q = S.f32_to_bf16_bits(rng.standard_normal((1, Hq, N, d)).astype(np.float32))
+    K = S.f32_to_bf16_bits(rng.standard_normal((1, Hkv, N, d)).astype(np.float32))
+    V = S.f32_to_bf16_bits(rng.standard_normal((1, Hkv, N, d)).astype(np.float32))
+    n_kb, n_qt = N // bk, N // tile_q
+    scores = O.block_scores(Q, K, tile_q, bk)
+    r = O.select(scores, tile_q, bk, n_kb, n_kb, 1, 0.25)
+    scale = 1.0 / math.sqrt(d)
+    out, lse = O.attend(Q, K, V, r["kv_idx"], tile_q, bk, scale)
+    for h in range(Hq):
+        ref = _sdpa(Q[0, h], K[0, h // 2], V[0, h // 2], scale)
+        np.testing.assert_allclose(out[0, h], ref, atol=1e-12, rtol=1e-10)
+        np.testing.assert_allclose(out[0, h], O.dense_causal_attention(
+            Q[0, h], K[0, h // 2], V[0, h // 2], scale), atol=1e-12)
+        # lse: log of the causal softmax denominator, by direct summation
+        qf, kf = O.widen(Q[0, h]), O.widen(K[0, h // 2])
+        lg = scale * qf @ kf.T
+        lg[np.triu(np.ones((N, N), bool), 1)] = -np.inf
+        np.testing.assert_allclose(lse[0, h], np.log(np.exp(lg).sum(axis=1)), rtol=1e-12)
+
+
+def test_attend_permutation_invariant():
+    rng = np.random.default_rng(9)
+    N, d, tile_q, bk = 512, 16, 64, 32
+    Q = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    K = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    V = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    s = O.block_scores(Q, K, tile_q, bk)
+    r = O.select(s, tile_q, bk, 6, 6, 1, 0.25)
+    kv = r["kv_idx"].copy()
+    out1, _ = O.attend(Q, K, V, kv, tile_q, bk, 0.25)
+    perm = kv.copy()
+    for t in range(kv.shape[2]):
+        c = r["kv_cnt"][0, 0, t]
+        perm[0, 0, t, :c] = rng.permutation(kv[0, 0, t, :c])
+    out2, _ = O.attend(Q, K, V, perm, tile_q, bk, 0.25)
+    np.testing.assert_allclose(out1, out2, atol=1e-12)
+
+
+def test_attend_sparse_matches_masked_dense():
+    """A sparse row equals dense attention with the unselected blocks masked out."""
+    rng = np.random.default_rng(10)
+    N, d, tile_q, bk = 256, 16, 32, 32
+    Q = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    K = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    V = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    s = O.block_scores(Q, K, tile_q, bk)
+    r = O.select(s, tile_q, bk, 3, 3, 1, 0.25)
+    out, _ = O.attend(Q, K, V, r["kv_idx"], tile_q, bk, 0.5)
+    q = torch.from_numpy(Q[0, 0].astype(np.float64))
+    k = torch.from_numpy(K[0, 0].astype(np.float64))
+    v = torch.from_numpy(V[0, 0].astype(np.float64))
+    mask = torch.zeros(N, N, dtype=torch.bool)
+    for t in range(N // tile_q):
+        for j in r["kv_idx"][0, 0, t]:
+            if j >= 0:
+                mask[t * tile_q:(t + 1) * tile_q, j * bk:(j + 1) * bk] = True
+    mask &= torch.ones(N, N, dtype=torch.bool).tril()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q[None, None], k[None, None], v[None, None], attn_mask=mask[None, None], scale=0.5)[0, 0]
+    np.testing.assert_allclose(out[0, 0], ref.numpy(), atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# decode: termination rule (hand-worked traces) and limits
+
+def _load_art(golden_dir):
+    cases, cur = [], None
+    for line in open(os.path.join(golden_dir, "art_decision.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        p = line.split()
+        if p[0] == "case":
+            cur = dict(name=p[1], tau=float(p[2]), phi=float(p[3]), p=int(p[4]),
+                       exp=int(p[5]), x=[])
+            cases.append(cur)
+        else:
+            cur["x"].append([float(v) for v in p[1:]])
+    return cases
+
+
+def test_termination_golden(golden_dir):
+    cases = _load_art(golden_dir)
+    assert len(cases) == 7
+    for c in cases:
+        tr = np.array(c["x"], np.float32)
+        assert O.termination_block(tr, c["tau"], c["phi"], c["p"]) == c["exp"], c["name"]
+
+
+def test_probe_step_values():
+    ds, dd = O.probe_step([3.0, 4.0], [6.0, 8.0])
+    assert ds == 5.0 and abs(dd) < 1e-15
+    ds, dd = O.probe_step([1.0, 0.0], [0.0, 2.0])
+    assert ds == 1.0 and dd == 1.0
+    ds, dd = O.probe_step([1.0, 0.0], [-1.0, 0.0])
+    assert ds == 0.0 and dd == 2.0
+
+
+def _decode_case(seed=11, L=2048, d=128, G=4, bkv=128):
+    rng = np.random.default_rng(seed)
+    q = S.f32_to_bf16_bits(rng.standard_normal((G, d)).astype(np.float32))
+    Kc = S.f32_to_bf16_bits(rng.standard_normal((L, d)).astype(np.float32))
+    Vc = S.f32_to_bf16_bits(rng.standard_normal((L, d)).astype(np.float32))
+    return q, Kc, Vc
+
+
+def test_decode_no_termination_is_dense():
+    q, Kc, Vc = _decode_case()
+    dims = S.default_probe_dims(32)
+    scale = 1 / math.sqrt(128)
+    o, used, tr = O.decode_group(q, Kc, Vc, 128, scale, 0.0, 0.0, 1, dims)
+    assert used == 16 and tr.shape == (16, 32)
+    qq = torch.from_numpy(O.widen(q))[None, :, None, :]
+    kk = torch.from_numpy(O.widen(Kc))[None, None].expand(1, 4, -1, -1)
+    vv = torch.from_numpy(O.widen(Vc))[None, None].expand(1, 4, -1, -1)
+    ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=scale)[0, :, 0]
+    np.testing.assert_allclose(o, ref.numpy(), atol=1e-12)
+
+
+@pytest.mark.parametrize("p", [1, 2, 5])
+def test_decode_infinite_thresholds_stop_after_p_plus_one(p):
+    q, Kc, Vc = _decode_case()
+    o, used, tr = O.decode_group(q, Kc, Vc, 128, 0.125, np.inf, np.inf, p, S.default_probe_dims())
+    assert used == p + 1
+    # the output is attention over exactly the first used*128 keys
+    n = used * 128
+    qq = torch.from_numpy(O.widen(q))[None, :, None, :]
+    kk = torch.from_numpy(O.widen(Kc[:n]))[None, None].expand(1, 4, -1, -1)
+    vv = torch.from_numpy(O.widen(Vc[:n]))[None, None].expand(1, 4, -1, -1)
+    ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=0.125)[0, :, 0]
+    np.testing.assert_allclose(o, ref.numpy(), atol=1e-12)
+
+
+def test_decode_planted_convergence():
+    """Keys of block 0 align with the query (huge logits), later keys point
+    away: the output is fixed after block 0, so the first test (t = 1) is
+    stable and streaming stops with 2 blocks."""
+    q, Kc, Vc = _decode_case()
+    qf = O.widen(q)[0]
+    Kf = np.tile(-qf, (2048, 1))
+    Kf[:128] = 4 * qf
+    Kb = S.f32_to_bf16_bits(Kf.astype(np.float32))
+    qb = np.tile(q[0], (4, 1))
+    o, used, tr = O.decode_group(qb, Kb, Vc, 128, 0.125, 1e-3, 1e-4, 1, S.default_probe_dims())
+    assert used == 2
+
+
+def test_generator_structure():
+    """The seeded generators plant the stated structure (not method arithmetic)."""
+    spec = S.WORKLOADS["gated_prefill_128k"].scaled(N=4096, Hq=4, Hkv=1)
+    k = S.prefill_head(spec, 1002, "k", 0, 0).reshape(-1, 64, 128)
+    twins = sum(np.array_equal(k[2 * m], k[2 * m + 1]) for m in range(32))
+    near = sum((k[2 * m] != k[2 * m + 1]).sum() == 1 for m in range(32))
+    assert twins + near >= 3
+    d = S.DECODE_WORKLOADS["decode_art_64k"].scaled(L=8192)
+    kk = S.bf16_bits_to_f32(S.decode_head(d, 1004, "k", 0, 0))
+    assert 1.6 < kk[:4096].std() / kk[4096:].std() < 2.4
+    a = S.prefill_head(spec, 5, "q", 0, 3)
+    b = S.prefill_head(spec, 5, "q", 0, 3)
+    assert np.array_equal(a, b)
