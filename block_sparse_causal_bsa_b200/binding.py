@@ -1,0 +1,267 @@
+"""ctypes binding of libbsa.so (the C ABI in include/bsa.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current stream. There is no CPU
+fallback; if the library is missing or fails to load, calls raise.
+
+The raw entry points keep the C names (``bsa_score``, ``bsa_select``,
+``bsa_attend``, ``bsa_decode`` and the sizing helpers) and take torch tensors
+or raw pointers; ``score``/``select``/``attend``/``decode``/``prefill`` allocate
+outputs with torch and call them.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbsa.so")
+
+BSA_OK, BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA = 0, 1, 2, 3
+BSA_DEV_OK, BSA_DEV_BAD_INDEX, BSA_DEV_TIMEOUT, BSA_DEV_BAD_SCORE = 0, 1, 2, 4
+BSA_BF16, BSA_F32 = 0, 1
+BSA_SCORE_MEAN, BSA_SCORE_MEAN_VNORM = 0, 1
+
+EXPORTS = ("bsa_score_workspace_bytes", "bsa_score", "bsa_kv_idx_width",
+           "bsa_select_workspace_bytes", "bsa_select", "bsa_attend", "bsa_decode",
+           "bsa_status_string", "bsa_last_error")
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"libbsa status {status}: {msg}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("N", ctypes.c_int), ("d", ctypes.c_int), ("block_k", ctypes.c_int),
+                ("tile_q", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class SelectParams(ctypes.Structure):
+    _fields_ = [("k_first", ctypes.c_int), ("k_last", ctypes.c_int), ("rho", ctypes.c_int),
+                ("gate_quantile", ctypes.c_float), ("gate_threshold", ctypes.c_float)]
+
+
+class DecodeShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("L", ctypes.c_int), ("d", ctypes.c_int), ("block_kv", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+class DecodeParams(ctypes.Structure):
+    _fields_ = [("tau", ctypes.c_float), ("phi", ctypes.c_float), ("patience", ctypes.c_int),
+                ("enable", ctypes.c_int), ("n_probe", ctypes.c_int),
+                ("probe_dims", ctypes.POINTER(ctypes.c_int))]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbsa.so (built by ``block_sparse_causal_bsa_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run python -m block_sparse_causal_bsa_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32p, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t
+        sp, pp = ctypes.POINTER(Shape), ctypes.POINTER(SelectParams)
+        dsp, dpp = ctypes.POINTER(DecodeShape), ctypes.POINTER(DecodeParams)
+        L.bsa_score_workspace_bytes.argtypes = [sp, ctypes.c_int]
+        L.bsa_score_workspace_bytes.restype = sz
+        L.bsa_score.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, vp, sz, vp]
+        L.bsa_score.restype = ctypes.c_int
+        L.bsa_kv_idx_width.argtypes = [sp, pp]
+        L.bsa_kv_idx_width.restype = ctypes.c_int
+        L.bsa_select_workspace_bytes.argtypes = [sp, pp]
+        L.bsa_select_workspace_bytes.restype = sz
+        L.bsa_select.argtypes = [sp, pp, vp, i32p, i32p, vp, vp, vp, vp, i32p, vp, sz, vp]
+        L.bsa_select.restype = ctypes.c_int
+        L.bsa_attend.argtypes = [sp, vp, vp, vp, i32p, i32p, ctypes.c_int, ctypes.c_float, vp, vp,
+                                 i32p, vp]
+        L.bsa_attend.restype = ctypes.c_int
+        L.bsa_decode.argtypes = [dsp, dpp, vp, vp, vp, ctypes.c_float, vp, i32p, vp, i32p, vp]
+        L.bsa_decode.restype = ctypes.c_int
+        L.bsa_status_string.argtypes = [ctypes.c_int]
+        L.bsa_status_string.restype = ctypes.c_char_p
+        L.bsa_last_error.argtypes = []
+        L.bsa_last_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != BSA_OK:
+        raise BsaError(status, lib().bsa_last_error().decode())
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BSA_BF16
+    if t.dtype == torch.float32:
+        return BSA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+@dataclasses.dataclass
+class SelectConfig:
+    """Selection parameters (mirrors bsa_select_params)."""
+    k_first: int
+    k_last: Optional[int] = None
+    rho: int = 1
+    gate_quantile: float = 0.25
+    gate_threshold: float = float("nan")
+
+    def c(self) -> SelectParams:
+        kl = self.k_first if self.k_last is None else self.k_last
+        return SelectParams(self.k_first, kl, self.rho, self.gate_quantile, self.gate_threshold)
+
+
+def make_shape(q: torch.Tensor, k: torch.Tensor, block_k: int, tile_q: int) -> Shape:
+    B, Hq, N, d = q.shape
+    return Shape(B, Hq, k.shape[1], N, d, block_k, tile_q, _dtype_code(q))
+
+
+# ---------------------------------------------------------------------------
+# raw entry points (C names)
+
+def bsa_score_workspace_bytes(shape: Shape, kind: int) -> int:
+    return lib().bsa_score_workspace_bytes(ctypes.byref(shape), kind)
+
+
+def bsa_score(shape, kind, q, k, v, scores, ws, ws_bytes, stream=None) -> None:
+    _check(lib().bsa_score(ctypes.byref(shape), kind, _ptr(q), _ptr(k), _ptr(v), _ptr(scores),
+                           _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def bsa_kv_idx_width(shape: Shape, params: SelectParams) -> int:
+    return lib().bsa_kv_idx_width(ctypes.byref(shape), ctypes.byref(params))
+
+
+def bsa_select_workspace_bytes(shape: Shape, params: SelectParams) -> int:
+    return lib().bsa_select_workspace_bytes(ctypes.byref(shape), ctypes.byref(params))
+
+
+def bsa_select(shape, params, scores, kv_idx, kv_cnt, sigma, sigma_bar, trigger, theta,
+               dev_status, ws, ws_bytes, stream=None) -> None:
+    _check(lib().bsa_select(ctypes.byref(shape), ctypes.byref(params), _ptr(scores), _ptr(kv_idx),
+                            _ptr(kv_cnt), _ptr(sigma), _ptr(sigma_bar), _ptr(trigger), _ptr(theta),
+                            _ptr(dev_status), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def bsa_attend(shape, q, k, v, kv_idx, kv_cnt, W, scale, out, lse, dev_status, stream=None) -> None:
+    _check(lib().bsa_attend(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_idx),
+                            _ptr(kv_cnt), W, scale, _ptr(out), _ptr(lse), _ptr(dev_status),
+                            _stream(stream)))
+
+
+def bsa_decode(shape, params, q, k_cache, v_cache, scale, out, blocks_used, probe_trace,
+               dev_status, stream=None) -> None:
+    _check(lib().bsa_decode(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k_cache),
+                            _ptr(v_cache), scale, _ptr(out), _ptr(blocks_used), _ptr(probe_trace),
+                            _ptr(dev_status), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# convenience wrappers (torch allocation + the raw calls)
+
+def _empty_bytes(n: int, device) -> torch.Tensor:
+    return torch.empty(max(int(n), 256), dtype=torch.uint8, device=device)
+
+
+def score(q, k, v=None, *, block_k: int, tile_q: int, output_aware: bool = False, stream=None):
+    shape = make_shape(q, k, block_k, tile_q)
+    kind = BSA_SCORE_MEAN_VNORM if output_aware else BSA_SCORE_MEAN
+    B, Hq, N, _ = q.shape
+    scores = torch.empty(B, Hq, N // tile_q, N // block_k, dtype=torch.float32, device=q.device)
+    nb = bsa_score_workspace_bytes(shape, kind)
+    ws = _empty_bytes(nb, q.device)
+    bsa_score(shape, kind, q, k, v if output_aware else None, scores, ws, nb, stream)
+    return scores
+
+
+def select(scores, *, shape: Shape, cfg: SelectConfig, stream=None):
+    dev = scores.device
+    p = cfg.c()
+    W = bsa_kv_idx_width(shape, p)
+    if W < 0:
+        raise BsaError(BSA_ERR_INVALID_ARG, lib().bsa_last_error().decode())
+    B, Hq, n_qt, _ = scores.shape
+    r = dict(
+        kv_idx=torch.empty(B, Hq, n_qt, W, dtype=torch.int32, device=dev),
+        kv_cnt=torch.empty(B, Hq, n_qt, dtype=torch.int32, device=dev),
+        sigma=torch.empty(B, Hq, n_qt, dtype=torch.float32, device=dev),
+        sigma_bar=torch.empty(B, n_qt, dtype=torch.float32, device=dev),
+        trigger=torch.empty(B, n_qt, dtype=torch.uint8, device=dev),
+        theta=torch.empty(1, dtype=torch.float32, device=dev),
+        dev_status=torch.zeros(1, dtype=torch.int32, device=dev),
+        W=W)
+    nb = bsa_select_workspace_bytes(shape, p)
+    ws = _empty_bytes(nb, dev)
+    bsa_select(shape, p, scores, r["kv_idx"], r["kv_cnt"], r["sigma"], r["sigma_bar"],
+               r["trigger"], r["theta"], r["dev_status"], ws, nb, stream)
+    return r
+
+
+def attend(q, k, v, kv_idx, kv_cnt, *, block_k: int, tile_q: int, scale: Optional[float] = None,
+           want_lse: bool = False, stream=None):
+    shape = make_shape(q, k, block_k, tile_q)
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
+    st = torch.zeros(1, dtype=torch.int32, device=q.device)
+    bsa_attend(shape, q, k, v, kv_idx, kv_cnt, kv_idx.shape[-1], scale, out, lse, st, stream)
+    return out, lse, st
+
+
+def decode(q, k_cache, v_cache, *, block_kv: int, tau: float, phi: float, patience: int = 1,
+           enable: bool = True, probe_dims: Sequence[int], scale: Optional[float] = None,
+           want_trace: bool = False, stream=None):
+    B, Hq, d = q.shape
+    Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    shape = DecodeShape(B, Hq, Hkv, L, d, block_kv, BSA_BF16)
+    dims = (ctypes.c_int * len(probe_dims))(*[int(x) for x in probe_dims])
+    params = DecodeParams(tau, phi, patience, int(enable), len(probe_dims), dims)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out = torch.empty_like(q)
+    used = torch.empty(B, Hkv, dtype=torch.int32, device=q.device)
+    trace = (torch.full((B, Hkv, L // block_kv, len(probe_dims)), float("nan"),
+                        dtype=torch.float32, device=q.device) if want_trace else None)
+    st = torch.zeros(1, dtype=torch.int32, device=q.device)
+    bsa_decode(shape, params, q, k_cache, v_cache, scale, out, used, trace, st, stream)
+    return out, used, trace, st
+
+
+def prefill(q, k, v, *, block_k: int, tile_q: int, cfg: SelectConfig, output_aware: bool = False,
+            scale: Optional[float] = None, stream=None):
+    """score -> select -> attend on the current stream; returns (out, selection dict, status)."""
+    shape = make_shape(q, k, block_k, tile_q)
+    s = score(q, k, v, block_k=block_k, tile_q=tile_q, output_aware=output_aware, stream=stream)
+    sel = select(s, shape=shape, cfg=cfg, stream=stream)
+    out, _, st = attend(q, k, v, sel["kv_idx"], sel["kv_cnt"], block_k=block_k, tile_q=tile_q,
+                        scale=scale, stream=stream)
+    sel["scores"] = s
+    return out, sel, st

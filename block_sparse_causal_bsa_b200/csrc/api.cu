@@ -1,0 +1,246 @@
+// C ABI of libbsa.so: argument validation, workspace layout and kernel dispatch.
+// Nothing here allocates device memory; every buffer is the caller's.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+bsa_status fail(bsa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bsa_status ok() {
+  g_err[0] = '\0';
+  return BSA_OK;
+}
+
+bsa_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(BSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bsa_status check_shape(const bsa_shape* s) {
+  if (!s) return fail(BSA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->N < 1)
+    return fail(BSA_ERR_INVALID_ARG, "B, Hq, Hkv, N must be >= 1");
+  if (s->Hq % s->Hkv) return fail(BSA_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+  if (s->d != 64 && s->d != 128) return fail(BSA_ERR_UNSUPPORTED, "d must be 64 or 128");
+  if ((s->block_k != 64 && s->block_k != 128) || (s->tile_q != 64 && s->tile_q != 128))
+    return fail(BSA_ERR_UNSUPPORTED, "block_k and tile_q must be 64 or 128");
+  if (s->N % s->block_k || s->N % s->tile_q)
+    return fail(BSA_ERR_INVALID_ARG, "N must be a multiple of block_k and tile_q");
+  if (s->dtype != BSA_BF16 && s->dtype != BSA_F32)
+    return fail(BSA_ERR_INVALID_ARG, "unknown dtype");
+  if ((long long)s->B * s->Hq * (s->N / s->tile_q) > (1ll << 31) - 1)
+    return fail(BSA_ERR_UNSUPPORTED, "too many query tiles");
+  return BSA_OK;
+}
+
+bsa_status check_params(const bsa_shape* s, const bsa_select_params* p) {
+  if (!p) return fail(BSA_ERR_INVALID_ARG, "params is NULL");
+  if (p->k_last < 1 || p->k_first < p->k_last)
+    return fail(BSA_ERR_INVALID_ARG, "need 1 <= k_last <= k_first");
+  if (p->rho < 1) return fail(BSA_ERR_INVALID_ARG, "rho must be >= 1");
+  if (!(p->gate_quantile <= 1.0f))
+    return fail(BSA_ERR_INVALID_ARG, "gate_quantile must be <= 1 (negative = fixed threshold)");
+  if (s->N / s->block_k > bsa::kMaxCandidates)
+    return fail(BSA_ERR_UNSUPPORTED, "more than %d key blocks", bsa::kMaxCandidates);
+  if ((long long)s->B * (s->N / s->tile_q) > bsa::kMaxGateTiles)
+    return fail(BSA_ERR_UNSUPPORTED, "B * n_qt above %d", bsa::kMaxGateTiles);
+  return BSA_OK;
+}
+
+struct ScoreWs {
+  float* kbar;
+  uint16_t* hi;
+  uint16_t* lo;
+  float* w;
+  size_t bytes;
+};
+
+ScoreWs score_ws(const bsa_shape& s, bsa_score_kind kind, void* base) {
+  const size_t nk = (size_t)s.B * s.Hkv * (s.N / s.block_k);
+  ScoreWs w{};
+  size_t off = 0;
+  char* p = (char*)base;
+  w.kbar = (float*)(p + off); off += align256(nk * s.d * 4);
+  w.hi = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
+  w.lo = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
+  w.w = (float*)(p + off); off += (kind == BSA_SCORE_MEAN_VNORM) ? align256(nk * 4) : 0;
+  if (kind != BSA_SCORE_MEAN_VNORM) w.w = nullptr;
+  w.bytes = off;
+  return w;
+}
+
+struct SelectWs {
+  int32_t* ranked;
+  float* sigma;
+  float* sigma_bar;
+  uint8_t* trigger;
+  size_t bytes;
+};
+
+SelectWs select_ws(const bsa_shape& s, int W, void* base) {
+  const size_t rows = (size_t)s.B * s.Hq * (s.N / s.tile_q);
+  const size_t tiles = (size_t)s.B * (s.N / s.tile_q);
+  SelectWs w{};
+  size_t off = 0;
+  char* p = (char*)base;
+  w.ranked = (int32_t*)(p + off); off += align256(rows * W * 4);
+  w.sigma = (float*)(p + off); off += align256(rows * 4);
+  w.sigma_bar = (float*)(p + off); off += align256(tiles * 4);
+  w.trigger = (uint8_t*)(p + off); off += align256(tiles);
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bsa_status_string(bsa_status st) {
+  switch (st) {
+    case BSA_OK: return "ok";
+    case BSA_ERR_INVALID_ARG: return "invalid argument";
+    case BSA_ERR_UNSUPPORTED: return "unsupported";
+    case BSA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* bsa_last_error(void) { return g_err; }
+
+size_t bsa_score_workspace_bytes(const bsa_shape* s, bsa_score_kind kind) {
+  if (check_shape(s) != BSA_OK) return 0;
+  return score_ws(*s, kind, nullptr).bytes;
+}
+
+bsa_status bsa_score(const bsa_shape* s, bsa_score_kind kind, const void* q, const void* k,
+                     const void* v, float* scores, void* ws, size_t ws_bytes, void* stream) {
+  bsa_status st = check_shape(s);
+  if (st != BSA_OK) return st;
+  if (kind != BSA_SCORE_MEAN && kind != BSA_SCORE_MEAN_VNORM)
+    return fail(BSA_ERR_INVALID_ARG, "unknown score kind");
+  if (!q || !k || !scores || !ws) return fail(BSA_ERR_INVALID_ARG, "NULL q, k, scores or workspace");
+  if (kind == BSA_SCORE_MEAN_VNORM && !v) return fail(BSA_ERR_INVALID_ARG, "v is NULL for VNORM");
+  if (!aligned16(q) || !aligned16(k) || (v && !aligned16(v)) || ((uintptr_t)ws & 255u))
+    return fail(BSA_ERR_INVALID_ARG, "q/k/v need 16-byte and workspace 256-byte alignment");
+  ScoreWs w = score_ws(*s, kind, ws);
+  if (ws_bytes < w.bytes) return fail(BSA_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, w.bytes);
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = bsa::launch_pool(*s, k, kind == BSA_SCORE_MEAN_VNORM ? v : nullptr, w.kbar,
+                                   s->dtype == BSA_BF16 ? w.hi : nullptr, w.lo, w.w, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "pool");
+  e = bsa::launch_score_simt(*s, q, w.kbar, w.w, scores, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "score");
+  return ok();
+}
+
+int bsa_kv_idx_width(const bsa_shape* s, const bsa_select_params* p) {
+  if (check_shape(s) != BSA_OK || check_params(s, p) != BSA_OK) return -1;
+  return bsa::kv_width(s->N, s->tile_q, s->block_k, p->k_first, p->k_last, p->rho);
+}
+
+size_t bsa_select_workspace_bytes(const bsa_shape* s, const bsa_select_params* p) {
+  if (check_shape(s) != BSA_OK || check_params(s, p) != BSA_OK) return 0;
+  int W = bsa::kv_width(s->N, s->tile_q, s->block_k, p->k_first, p->k_last, p->rho);
+  return select_ws(*s, W, nullptr).bytes;
+}
+
+bsa_status bsa_select(const bsa_shape* s, const bsa_select_params* p, const float* scores,
+                      int32_t* kv_idx, int32_t* kv_cnt, float* sigma, float* sigma_bar,
+                      uint8_t* trigger, float* theta, int32_t* dev_status, void* ws,
+                      size_t ws_bytes, void* stream) {
+  bsa_status st = check_shape(s);
+  if (st != BSA_OK) return st;
+  st = check_params(s, p);
+  if (st != BSA_OK) return st;
+  if (!scores || !kv_idx || !kv_cnt || !ws)
+    return fail(BSA_ERR_INVALID_ARG, "NULL scores, kv_idx, kv_cnt or workspace");
+  if ((uintptr_t)ws & 255u) return fail(BSA_ERR_INVALID_ARG, "workspace needs 256-byte alignment");
+  const int W = bsa::kv_width(s->N, s->tile_q, s->block_k, p->k_first, p->k_last, p->rho);
+  SelectWs w = select_ws(*s, W, ws);
+  if (ws_bytes < w.bytes) return fail(BSA_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, w.bytes);
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e;
+  if (dev_status) {
+    e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
+  }
+  float* sg = sigma ? sigma : w.sigma;
+  float* sb = sigma_bar ? sigma_bar : w.sigma_bar;
+  uint8_t* tr = trigger ? trigger : w.trigger;
+  e = bsa::launch_select_rank(*s, *p, scores, W, w.ranked, sg, dev_status, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "select_rank");
+  e = bsa::launch_gate(*s, *p, sg, sb, tr, theta, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "gate");
+  e = bsa::launch_finalize(*s, *p, w.ranked, W, tr, W, kv_idx, kv_cnt, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "finalize");
+  return ok();
+}
+
+bsa_status bsa_attend(const bsa_shape* s, const void* q, const void* k, const void* v,
+                      const int32_t* kv_idx, const int32_t* kv_cnt, int W, float scale, void* out,
+                      float* lse, int32_t* dev_status, void* stream) {
+  bsa_status st = check_shape(s);
+  if (st != BSA_OK) return st;
+  if (!q || !k || !v || !kv_idx || !kv_cnt || !out || !dev_status)
+    return fail(BSA_ERR_INVALID_ARG, "NULL q, k, v, kv_idx, kv_cnt, out or dev_status");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(BSA_ERR_INVALID_ARG, "q/k/v/out need 16-byte alignment");
+  if (W < 1 || W > s->N / s->block_k) return fail(BSA_ERR_INVALID_ARG, "W out of range");
+  if (!(scale > 0.0f)) return fail(BSA_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
+  e = bsa::launch_attend_simt(*s, q, k, v, kv_idx, kv_cnt, W, scale, out, lse, dev_status, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "attend");
+  return ok();
+}
+
+bsa_status bsa_decode(const bsa_decode_shape* s, const bsa_decode_params* p, const void* q,
+                      const void* kc, const void* vc, float scale, void* out, int32_t* blocks_used,
+                      float* probe_trace, int32_t* dev_status, void* stream) {
+  if (!s || !p) return fail(BSA_ERR_INVALID_ARG, "shape or params is NULL");
+  if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->L < 1 || s->Hq % s->Hkv)
+    return fail(BSA_ERR_INVALID_ARG, "bad B/Hq/Hkv/L");
+  const int G = s->Hq / s->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(BSA_ERR_UNSUPPORTED, "Hq/Hkv must be 1, 2, 4 or 8");
+  if (s->d != 64 && s->d != 128) return fail(BSA_ERR_UNSUPPORTED, "d must be 64 or 128");
+  if (s->block_kv != 64 && s->block_kv != 128) return fail(BSA_ERR_UNSUPPORTED, "block_kv must be 64 or 128");
+  if (s->L % s->block_kv) return fail(BSA_ERR_INVALID_ARG, "L must be a multiple of block_kv");
+  if (s->dtype != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "decode takes bf16 only");
+  if (p->patience < 1) return fail(BSA_ERR_INVALID_ARG, "patience must be >= 1");
+  if (p->n_probe < 1 || p->n_probe > bsa::kMaxProbe || !p->probe_dims)
+    return fail(BSA_ERR_INVALID_ARG, "n_probe must be 1..%d with probe_dims given", bsa::kMaxProbe);
+  for (int i = 0; i < p->n_probe; ++i)
+    if (p->probe_dims[i] < 0 || p->probe_dims[i] >= s->d)
+      return fail(BSA_ERR_INVALID_ARG, "probe_dims[%d] out of range", i);
+  if (!(p->tau >= 0.0f) || !(p->phi >= 0.0f)) return fail(BSA_ERR_INVALID_ARG, "tau and phi must be >= 0");
+  if (!q || !kc || !vc || !out || !blocks_used || !dev_status)
+    return fail(BSA_ERR_INVALID_ARG, "NULL q, caches, out, blocks_used or dev_status");
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(out))
+    return fail(BSA_ERR_INVALID_ARG, "q/caches/out need 16-byte alignment");
+  if (!(scale > 0.0f)) return fail(BSA_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
+  e = bsa::launch_decode(*s, *p, q, kc, vc, scale, out, blocks_used, probe_trace, dev_status, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "decode");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Internal launchers behind the C ABI (host side). Each returns cudaError_t of the launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/bsa.h"
+
+namespace bsa {
+
+// Pooled keys (+ value-block norms). kbar fp32 [B,Hkv,n_kb,d]; kbar_hi/lo bf16 split of
+// kbar (may be null); wnorm [B,Hkv,n_kb] (only when v != null).
+cudaError_t launch_pool(const bsa_shape& s, const void* k, const void* v, float* kbar,
+                        uint16_t* kbar_hi, uint16_t* kbar_lo, float* wnorm, cudaStream_t st);
+
+// Block scores on CUDA cores (fp32 FMA).
+cudaError_t launch_score_simt(const bsa_shape& s, const void* q, const float* kbar,
+                              const float* wnorm, float* scores, cudaStream_t st);
+
+// Block scores on tcgen05 tensor cores (bf16 inputs, hi/lo split of the pooled keys).
+cudaError_t launch_score_tc(const bsa_shape& s, const void* q, const uint16_t* kbar_hi,
+                            const uint16_t* kbar_lo, const float* wnorm, float* scores,
+                            int32_t* dev_status, cudaStream_t st);
+
+// Selection: ranked candidate lists + sigma, then the gate, then kv_idx.
+cudaError_t launch_select_rank(const bsa_shape& s, const bsa_select_params& p, const float* scores,
+                               int R, int32_t* ranked, float* sigma, int32_t* dev_status,
+                               cudaStream_t st);
+cudaError_t launch_gate(const bsa_shape& s, const bsa_select_params& p, const float* sigma,
+                        float* sigma_bar, uint8_t* trigger, float* theta, cudaStream_t st);
+cudaError_t launch_finalize(const bsa_shape& s, const bsa_select_params& p, const int32_t* ranked,
+                            int R, const uint8_t* trigger, int W, int32_t* kv_idx, int32_t* kv_cnt,
+                            cudaStream_t st);
+
+// Sparse attend on CUDA cores (fp32 math; bf16 or fp32 I/O).
+cudaError_t launch_attend_simt(const bsa_shape& s, const void* q, const void* k, const void* v,
+                               const int32_t* kv_idx, const int32_t* kv_cnt, int W, float scale,
+                               void* out, float* lse, int32_t* dev_status, cudaStream_t st);
+
+// Sparse attend on tcgen05 tensor cores (bf16, d = 128, block_k = 64, tile_q = 128).
+bool attend_tc_supported(const bsa_shape& s);
+cudaError_t launch_attend_tc(const bsa_shape& s, const void* q, const void* k, const void* v,
+                             const int32_t* kv_idx, const int32_t* kv_cnt, int W, float scale,
+                             void* out, float* lse, int32_t* dev_status, cudaStream_t st);
+
+// Decode with run-time termination.
+cudaError_t launch_decode(const bsa_decode_shape& s, const bsa_decode_params& p, const void* q,
+                          const void* kc, const void* vc, float scale, void* out,
+                          int32_t* blocks_used, float* probe_trace, int32_t* dev_status,
+                          cudaStream_t st);
+
+// Limits of this build (checked on the host).
+constexpr int kMaxCandidates = 8192;     // n_kb for the in-shared-memory ranking sort
+constexpr int kMaxGateTiles = 16384;     // B * n_qt for the single-CTA gate sort
+constexpr int kMaxProbe = 64;
+constexpr int kMaxGroup = 8;             // Hq / Hkv in decode
+
+}  // namespace bsa

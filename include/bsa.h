@@ -1,0 +1,205 @@
+/*
+ * bsa.h -- C ABI of libbsa.so: block-sparse causal attention on NVIDIA B200 (sm_100a).
+ *
+ * Pages the operations follow (cited by title and section):
+ *   [UGS]  "Resumo Técnico: Seleção com Portão de Incerteza para Atenção de
+ *          Esparsidade em Blocos", Metodologia steps 1-5.
+ *   [Stem] "Stem: Rethinking Causal Information Flow in Sparse Attention",
+ *          Resumo técnico, 2. Metodologia A (TPD), B (OAM), Implementação.
+ *   [ART]  "Resumo Técnico: ART (Attention Run-time Termination)", 2. Metodologia 2.1-2.4.
+ *
+ * The problem as those pages frame it: block scores -> per-tile top-k list
+ * kv_idx -> sparse attention that streams only the listed blocks ([UGS] steps
+ * 2 and 5); and for decode: stream KV blocks in order and stop once the
+ * partial output is stable ([ART] 2.2, 2.3).
+ *
+ * Conventions shared by every call
+ *   Layout     Q [B,Hq,N,d], K and V [B,Hkv,N,d], O like Q; contiguous, d innermost.
+ *              Query head h reads KV head h / (Hq/Hkv).
+ *   Tiles      query tile t = rows [t*tile_q, (t+1)*tile_q); key block j = keys
+ *              [j*block_k, (j+1)*block_k); n_qt = N/tile_q, n_kb = N/block_k.
+ *              Causal: query i sees keys 0..i. J_t = ((t+1)*tile_q-1)/block_k is
+ *              the last block tile t can see; blocks (t*tile_q)/block_k .. J_t
+ *              intersect the tile's own rows and are always kept ("forced").
+ *   Memory     Every tensor argument is a DEVICE pointer owned by the caller,
+ *              unless a comment says "host". The library never allocates or
+ *              frees; workspace is caller-provided and sized by the *_bytes calls.
+ *   Streams    `stream` is a cudaStream_t (NULL = legacy default stream). All
+ *              compute calls only enqueue work and return; results are ready
+ *              after the stream is synchronised.
+ *   Errors     Argument errors are detected on the host before anything is
+ *              enqueued and return BSA_ERR_INVALID_ARG / BSA_ERR_UNSUPPORTED;
+ *              launch failures return BSA_ERR_CUDA. bsa_last_error() gives a
+ *              one-line reason (per thread). Problems only the device can see
+ *              (an out-of-range kv_idx entry, a non-finite candidate score, a
+ *              wait that ran out) are OR-ed into *dev_status as BSA_DEV_* bits;
+ *              the call clears *dev_status first, the offending work is
+ *              skipped, and the kernel never traps.
+ *   Precision  bf16 inputs, fp32 accumulation and softmax; BSA_F32 inputs run
+ *              an fp32 CUDA-core path.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, workspace too small, ... */
+  BSA_ERR_UNSUPPORTED = 2,   /* valid but outside what this build implements */
+  BSA_ERR_CUDA = 3           /* a CUDA launch or runtime call failed */
+} bsa_status;
+
+/* Bits OR-ed into *dev_status by the device. */
+enum {
+  BSA_DEV_OK = 0,
+  BSA_DEV_BAD_INDEX = 1,     /* kv_idx entry >= n_kb, > J_t, or a count > W */
+  BSA_DEV_TIMEOUT = 2,       /* a bounded wait on an mbarrier ran out */
+  BSA_DEV_BAD_SCORE = 4      /* a candidate block score was NaN or infinite */
+};
+
+typedef enum { BSA_BF16 = 0, BSA_F32 = 1 } bsa_dtype;
+
+/* Block score backbone.
+ *   BSA_SCORE_MEAN        s(t,j) = max over the tile's rows i of q_i . mean(K block j)
+ *                         ([UGS] steps 1-2: mean-pooled keys, tile max over rows).
+ *   BSA_SCORE_MEAN_VNORM  the same max times || mean(V block j) ||_2, an output-aware
+ *                         weighting of the block (motivated by [Stem] 2.B: value
+ *                         magnitude enters the selection metric). */
+typedef enum { BSA_SCORE_MEAN = 0, BSA_SCORE_MEAN_VNORM = 1 } bsa_score_kind;
+
+/* Prefill problem. d in {64,128}; block_k, tile_q in {64,128}; N a multiple of both. */
+typedef struct {
+  int B, Hq, Hkv, N, d, block_k, tile_q;
+  bsa_dtype dtype;
+} bsa_shape;
+
+/* Selection parameters.
+ *   k_first, k_last  budget in blocks, counting the forced blocks. Equal = fixed
+ *                    top-k ([UGS] step 2). Otherwise the Token Position-Decay budget
+ *                    of [Stem] 2.A, read as the linear decay
+ *                    k_t = k_first - floor((k_first-k_last)*t/(n_qt-1)).
+ *                    Requires 1 <= k_last <= k_first. Every budget is capped at the
+ *                    J_t+1 blocks the tile can see and never drops the forced blocks.
+ *   rho              expansion factor for triggered tiles: top-rho*k instead of
+ *                    top-k ([UGS] step 5). rho = 1 disables the gate.
+ *   gate_quantile    q in [0,1]: theta = linear-interpolation empirical q-quantile of
+ *                    the head-mean sigma over the cut tiles of this call (one call =
+ *                    one layer, [UGS] step 4). A negative value selects the fixed
+ *                    gate_threshold instead.
+ *   gate_threshold   fixed theta when gate_quantile < 0. */
+typedef struct {
+  int k_first, k_last;
+  int rho;
+  float gate_quantile;
+  float gate_threshold;
+} bsa_select_params;
+
+/* Decode problem: one query token per sequence, KV cache of length L.
+ * d in {64,128}; block_kv in {64,128}; L a multiple of block_kv; Hq/Hkv <= 8. */
+typedef struct {
+  int B, Hq, Hkv, L, d, block_kv;
+  bsa_dtype dtype;           /* BSA_BF16 only */
+} bsa_decode_shape;
+
+/* Run-time termination ([ART] 2.2-2.4).
+ *   tau, phi     thresholds: block t >= 1 is stable iff |‖x_t‖-‖x_{t-1}‖| < tau and
+ *                1 - cos(x_t, x_{t-1}) < phi (1 when a norm is 0), computed in fp64
+ *                on the fp32 probe values with sums in index order.
+ *   patience     stop after `patience` consecutive stable blocks (>= 1) ([ART] 2.3).
+ *   enable       0 = never stop (probes are still recorded when asked for).
+ *   n_probe      number of probe coordinates (1..64).
+ *   probe_dims   HOST array of n_probe coordinates in [0,d): the probe x^(t) is the
+ *                normalised partial output O^(t) of the KV group's first query head
+ *                at these coordinates ([ART] 2.2 names a register fragment of the
+ *                leading thread; this build fixes a layout-free coordinate set). */
+typedef struct {
+  float tau, phi;
+  int patience;
+  int enable;
+  int n_probe;
+  const int* probe_dims;
+} bsa_decode_params;
+
+/* ---- scoring ([UGS] steps 1-2; [Stem] 2.B, Implementação) ------------------------ */
+
+/* Workspace bytes bsa_score needs (pooled keys and the value-block norms). */
+size_t bsa_score_workspace_bytes(const bsa_shape* shape, bsa_score_kind kind);
+
+/* scores [B,Hq,n_qt,n_kb] fp32: s(t,j) for j <= J_t, -inf for j > J_t.
+ * No 1/sqrt(d) factor (a common positive factor changes neither the ranking nor sigma).
+ * The tile max runs over all tile_q rows, unmasked.
+ * q, k: inputs of `shape->dtype`; v is read only for BSA_SCORE_MEAN_VNORM (else may be NULL). */
+bsa_status bsa_score(const bsa_shape* shape, bsa_score_kind kind,
+                     const void* q, const void* k, const void* v,
+                     float* scores, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- selection ([UGS] steps 2-5; [Stem] 2.A) -------------------------------------- */
+
+/* kv_idx row width W = min(n_kb, max(rho*max(k_first,k_last), forced blocks per tile)).
+ * Depends only on the parameters, never on data ([UGS] step 5: uniform dispatch shape).
+ * Returns -1 on invalid arguments. */
+int bsa_kv_idx_width(const bsa_shape* shape, const bsa_select_params* params);
+
+size_t bsa_select_workspace_bytes(const bsa_shape* shape, const bsa_select_params* params);
+
+/* From scores (as written by bsa_score, same stream) to kv_idx.
+ *   kv_idx   [B,Hq,n_qt,W] int32: the forced blocks plus the best m_t (or, for a
+ *            triggered tile, M_t) candidate blocks, ranked by (score desc, index asc),
+ *            written in ascending order and padded with -1 ([UGS] steps 2, 5).
+ *   kv_cnt   [B,Hq,n_qt] int32: number of valid entries.
+ *   sigma    [B,Hq,n_qt] fp32 or NULL: (s_(m-1)-s_(m))/(s_(0)-s_(m)) over the ranked
+ *            candidates with m = m_t, fp32 ([UGS] step 3); 1 for a tile with no cut.
+ *   sigma_bar[B,n_qt] fp32 or NULL: fp32 head sum in head order, / Hq ([UGS] step 4).
+ *   trigger  [B,n_qt] uint8 or NULL: cut tile and sigma_bar < theta (strict).
+ *   theta    device fp32 scalar or NULL (NaN when undefined).
+ *   dev_status device int32 or NULL: BSA_DEV_BAD_SCORE on a non-finite candidate. */
+bsa_status bsa_select(const bsa_shape* shape, const bsa_select_params* params,
+                      const float* scores, int32_t* kv_idx, int32_t* kv_cnt,
+                      float* sigma, float* sigma_bar, uint8_t* trigger, float* theta,
+                      int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* ---- sparse attend ([UGS] step 5; [Stem] Implementação) ------------------------- */
+
+/* O_i = sum over keys j in the listed blocks with j <= i of softmax(scale * q_i.k_j) v_j.
+ *   kv_idx/kv_cnt as written by bsa_select (entries beyond kv_cnt ignored; order free).
+ *   out  like Q, of `shape->dtype`.  lse [B,Hq,N] fp32 or NULL: natural log of the
+ *        softmax denominator (-inf for a row that sees no key; its output row is 0).
+ *   dev_status  device int32, required. */
+bsa_status bsa_attend(const bsa_shape* shape, const void* q, const void* k, const void* v,
+                      const int32_t* kv_idx, const int32_t* kv_cnt, int W, float softmax_scale,
+                      void* out, float* lse, int32_t* dev_status, void* stream);
+
+/* ---- decode with run-time termination ([ART] 2.1-2.4) ----------------------------- */
+
+/* q [B,Hq,d], k_cache/v_cache [B,Hkv,L,d] bf16. Per (batch, KV head) the blocks
+ * 0,1,2,... are streamed in order with an online softmax for the group's query heads;
+ * block 0 is always processed ([ART] 2.4); after each block t >= 1 the stability test
+ * runs and streaming stops after `patience` consecutive stable blocks.
+ *   out          [B,Hq,d] bf16: normalised output over the processed blocks.
+ *   blocks_used  [B,Hkv] int32.
+ *   probe_trace  [B,Hkv,L/block_kv,n_probe] fp32 or NULL: x^(t) for every processed
+ *                block (later entries untouched).
+ *   dev_status   device int32, required. */
+bsa_status bsa_decode(const bsa_decode_shape* shape, const bsa_decode_params* params,
+                      const void* q, const void* k_cache, const void* v_cache,
+                      float softmax_scale, void* out, int32_t* blocks_used,
+                      float* probe_trace, int32_t* dev_status, void* stream);
+
+/* ---- misc --------------------------------------------------------------------------- */
+
+const char* bsa_status_string(bsa_status status);
+/* Reason for the last non-OK status returned on this thread ("" if none). */
+const char* bsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */

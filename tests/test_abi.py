@@ -1,0 +1,134 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, and its host-side validation and sizing logic agree with the
+oracle's definitions. No compute call reaches a kernel here (every call below
+is rejected on the host before anything is enqueued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_causal_bsa_b200 import binding as bb
+from oracle import bsa_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "bsa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsa_[a-z_]+)\s*\(", txt)))
+
+
+def test_header_declares_expected_calls():
+    assert set(_declared()) == set(bb.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = bb.lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    L = bb.lib()
+    for st in range(4):
+        assert L.bsa_status_string(st)
+
+
+def _shape(**kw):
+    base = dict(B=1, Hq=32, Hkv=8, N=131072, d=128, block_k=64, tile_q=128, dtype=bb.BSA_BF16)
+    base.update(kw)
+    return bb.Shape(*[base[f] for f, _ in bb.Shape._fields_])
+
+
+@pytest.mark.parametrize("N,tq,bk,kf,kl,rho", [
+    (131072, 128, 64, 64, 64, 2), (1024, 64, 64, 4, 4, 1), (65536, 128, 64, 128, 32, 1),
+    (2048, 128, 64, 1, 1, 1), (4096, 64, 128, 8, 2, 3), (512, 128, 128, 100, 100, 1),
+    (32768, 128, 64, 64, 64, 1)])
+def test_kv_width_matches_oracle(N, tq, bk, kf, kl, rho):
+    s = _shape(N=N, tile_q=tq, block_k=bk)
+    p = bb.SelectParams(kf, kl, rho, 0.25, float("nan"))
+    assert bb.bsa_kv_idx_width(s, p) == O.kv_idx_width(N, tq, bk, kf, kl, rho)
+
+
+def test_workspace_sizes():
+    s = _shape()
+    n = bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_MEAN)
+    nkb = 8 * 2048
+    assert n >= nkb * 128 * (4 + 2 + 2)
+    n2 = bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_MEAN_VNORM)
+    assert n2 >= n + nkb * 4
+    p = bb.SelectParams(64, 64, 2, 0.25, float("nan"))
+    sel = bb.bsa_select_workspace_bytes(s, p)
+    assert sel >= 32 * 1024 * 128 * 4
+
+
+@pytest.mark.parametrize("bad", [
+    dict(d=96), dict(block_k=32), dict(tile_q=256), dict(N=1000), dict(Hq=6, Hkv=4),
+    dict(B=0), dict(dtype=7)])
+def test_bad_shapes_rejected(bad):
+    s = _shape(**bad)
+    L = bb.lib()
+    st = L.bsa_score(ctypes.byref(s), 0, 16, 16, None, 16, 256, 1 << 30, None)
+    assert st in (bb.BSA_ERR_INVALID_ARG, bb.BSA_ERR_UNSUPPORTED)
+    assert L.bsa_last_error()
+    p = bb.SelectParams(8, 8, 1, 0.25, 0.0)
+    assert bb.bsa_kv_idx_width(s, p) == -1
+    assert bb.bsa_score_workspace_bytes(s, 0) == 0
+
+
+def test_null_pointers_rejected():
+    L = bb.lib()
+    s = _shape()
+    assert L.bsa_score(ctypes.byref(s), 0, None, 16, None, 16, 256, 1 << 30, None) == bb.BSA_ERR_INVALID_ARG
+    # output-aware score without V
+    assert L.bsa_score(ctypes.byref(s), 1, 16, 16, None, 16, 256, 1 << 30, None) == bb.BSA_ERR_INVALID_ARG
+    # undersized workspace
+    assert L.bsa_score(ctypes.byref(s), 0, 16, 16, None, 16, 256, 10, None) == bb.BSA_ERR_INVALID_ARG
+    assert b"workspace" in L.bsa_last_error()
+    # misaligned pointer
+    assert L.bsa_score(ctypes.byref(s), 0, 18, 16, None, 16, 256, 1 << 30, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_attend(ctypes.byref(s), 16, 16, 16, 16, 16, 128, 0.1, 16, None, None, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_attend(ctypes.byref(s), 16, 16, 16, 16, 16, 0, 0.1, 16, None, 16, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_attend(ctypes.byref(s), 16, 16, 16, 16, 16, 128, -1.0, 16, None, 16, None) == bb.BSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kf,kl,rho,q", [(4, 8, 1, 0.2), (0, 0, 1, 0.2), (8, 8, 0, 0.2), (8, 8, 2, 1.5)])
+def test_bad_select_params_rejected(kf, kl, rho, q):
+    L = bb.lib()
+    s = _shape()
+    p = bb.SelectParams(kf, kl, rho, q, 0.0)
+    assert L.bsa_select(ctypes.byref(s), ctypes.byref(p), 16, 16, 16, None, None, None, None, None,
+                        256, 1 << 34, None) == bb.BSA_ERR_INVALID_ARG
+
+
+def test_select_size_limits():
+    L = bb.lib()
+    s = _shape(N=64 * 16384)      # more key blocks than the in-shared-memory sort takes
+    p = bb.SelectParams(8, 8, 1, 0.25, 0.0)
+    assert L.bsa_select(ctypes.byref(s), ctypes.byref(p), 16, 16, 16, None, None, None, None, None,
+                        256, 1 << 40, None) == bb.BSA_ERR_UNSUPPORTED
+
+
+def test_decode_validation():
+    L = bb.lib()
+    dims = (ctypes.c_int * 2)(0, 1)
+    ok_shape = bb.DecodeShape(2, 32, 8, 8192, 128, 128, bb.BSA_BF16)
+    p = bb.DecodeParams(1e-3, 1e-4, 1, 1, 2, dims)
+    # missing dev_status
+    assert L.bsa_decode(ctypes.byref(ok_shape), ctypes.byref(p), 16, 16, 16, 0.1, 16, 16, None,
+                        None, None) == bb.BSA_ERR_INVALID_ARG
+    for bad in [dict(L=8000), dict(Hq=24), dict(block_kv=32), dict(dtype=bb.BSA_F32)]:
+        f = dict(B=2, Hq=32, Hkv=8, L=8192, d=128, block_kv=128, dtype=bb.BSA_BF16)
+        f.update(bad)
+        sh = bb.DecodeShape(*[f[n] for n, _ in bb.DecodeShape._fields_])
+        assert L.bsa_decode(ctypes.byref(sh), ctypes.byref(p), 16, 16, 16, 0.1, 16, 16, None, 16,
+                            None) in (bb.BSA_ERR_INVALID_ARG, bb.BSA_ERR_UNSUPPORTED)
+    bad_dims = (ctypes.c_int * 2)(0, 128)
+    p2 = bb.DecodeParams(1e-3, 1e-4, 1, 1, 2, bad_dims)
+    assert L.bsa_decode(ctypes.byref(ok_shape), ctypes.byref(p2), 16, 16, 16, 0.1, 16, 16, None, 16,
+                        None) == bb.BSA_ERR_INVALID_ARG
+    p3 = bb.DecodeParams(1e-3, 1e-4, 0, 1, 2, dims)
+    assert L.bsa_decode(ctypes.byref(ok_shape), ctypes.byref(p3), 16, 16, 16, 0.1, 16, 16, None, 16,
+                        None) == bb.BSA_ERR_INVALID_ARG
