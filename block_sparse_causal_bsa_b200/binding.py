@@ -29,7 +29,8 @@ BSA_SCORE_MEAN, BSA_SCORE_MEAN_VNORM = 0, 1
 
 EXPORTS = ("bsa_score_workspace_bytes", "bsa_score", "bsa_kv_idx_width",
            "bsa_select_workspace_bytes", "bsa_select", "bsa_attend", "bsa_decode",
-           "bsa_status_string", "bsa_last_error")
+           "bsa_status_string", "bsa_last_error", "bsa_select_noalloc_max_bytes",
+           "bsa_select_noalloc")
 
 
 class BsaError(RuntimeError):
@@ -89,6 +90,10 @@ def lib() -> ctypes.CDLL:
         L.bsa_attend.restype = ctypes.c_int
         L.bsa_decode.argtypes = [dsp, dpp, vp, vp, vp, ctypes.c_float, vp, i32p, vp, i32p, vp]
         L.bsa_decode.restype = ctypes.c_int
+        L.bsa_select_noalloc_max_bytes.argtypes = []
+        L.bsa_select_noalloc_max_bytes.restype = sz
+        L.bsa_select_noalloc.argtypes = [sp, pp, vp, i32p, i32p, vp, vp, vp, vp, i32p, vp]
+        L.bsa_select_noalloc.restype = ctypes.c_int
         L.bsa_status_string.argtypes = [ctypes.c_int]
         L.bsa_status_string.restype = ctypes.c_char_p
         L.bsa_last_error.argtypes = []
@@ -170,6 +175,15 @@ def bsa_select(shape, params, scores, kv_idx, kv_cnt, sigma, sigma_bar, trigger,
     _check(lib().bsa_select(ctypes.byref(shape), ctypes.byref(params), _ptr(scores), _ptr(kv_idx),
                             _ptr(kv_cnt), _ptr(sigma), _ptr(sigma_bar), _ptr(trigger), _ptr(theta),
                             _ptr(dev_status), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def bsa_select_noalloc(shape, params, scores, kv_idx, kv_cnt, sigma, sigma_bar, trigger, theta,
+                       dev_status, stream=None) -> None:
+    """bsa_select with the library's static scratch instead of a workspace (no allocation)."""
+    _check(lib().bsa_select_noalloc(ctypes.byref(shape), ctypes.byref(params), _ptr(scores),
+                                    _ptr(kv_idx), _ptr(kv_cnt), _ptr(sigma), _ptr(sigma_bar),
+                                    _ptr(trigger), _ptr(theta), _ptr(dev_status),
+                                    _stream(stream)))
 
 
 def bsa_attend(shape, q, k, v, kv_idx, kv_cnt, W, scale, out, lse, dev_status, stream=None) -> None:

@@ -109,6 +109,15 @@ SelectWs select_ws(const bsa_shape& s, int W, void* base) {
 
 }  // namespace
 
+namespace bsa {
+void set_last_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+}  // namespace bsa
+
 extern "C" {
 
 const char* bsa_status_string(bsa_status st) {

@@ -49,6 +49,9 @@ cudaError_t launch_decode(const bsa_decode_shape& s, const bsa_decode_params& p,
                           int32_t* blocks_used, float* probe_trace, int32_t* dev_status,
                           cudaStream_t st);
 
+// Sets the text bsa_last_error() returns on this thread.
+void set_last_error(const char* fmt, ...);
+
 // Limits of this build (checked on the host).
 constexpr int kMaxCandidates = 8192;     // n_kb for the in-shared-memory ranking sort
 constexpr int kMaxGateTiles = 16384;     // B * n_qt for the single-CTA gate sort

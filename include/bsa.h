@@ -192,6 +192,28 @@ bsa_status bsa_decode(const bsa_decode_shape* shape, const bsa_decode_params* pa
                       float softmax_scale, void* out, int32_t* blocks_used,
                       float* probe_trace, int32_t* dev_status, void* stream);
 
+/* ---- selection without a caller-provided workspace -------------------------------- */
+
+/* The pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory (for example a plugin whose host process owns all device
+ * memory through its own pool, or a serving loop where a cudaMalloc could
+ * synchronise the device). It does exactly what bsa_select does, with the same
+ * arguments minus the workspace, and allocates nothing: its scratch is a static
+ * array of bsa_select_noalloc_max_bytes() bytes (32 MiB) in device memory that
+ * every GPU loading libbsa.so keeps until the process exits.
+ *   - Shapes whose bsa_select_workspace_bytes() exceed that size are rejected with
+ *     BSA_ERR_UNSUPPORTED (bsa_last_error() says why); nothing is launched.
+ *   - The first call on a device looks up the array's device address (with that
+ *     device current) and caches it; make that first call before any stream capture.
+ *   - All calls share the one array. Calls that overlap on the GPU (other streams,
+ *     other host threads on the same device) race on it: the caller must order them.
+ *     The array keeps the last call's contents; no entry has to start at zero. */
+size_t bsa_select_noalloc_max_bytes(void);
+bsa_status bsa_select_noalloc(const bsa_shape* shape, const bsa_select_params* params,
+                              const float* scores, int32_t* kv_idx, int32_t* kv_cnt,
+                              float* sigma, float* sigma_bar, uint8_t* trigger, float* theta,
+                              int32_t* dev_status, void* stream);
+
 /* ---- misc --------------------------------------------------------------------------- */
 
 const char* bsa_status_string(bsa_status status);
