@@ -215,8 +215,15 @@ bsa_status bsa_attend(const bsa_shape* s, const void* q, const void* k, const vo
   cudaStream_t cs = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
   if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
-  e = bsa::launch_attend_simt(*s, q, k, v, kv_idx, kv_cnt, W, scale, out, lse, dev_status, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "attend");
+  // tensor-core path for its shapes (bf16, d 128, blocks 64, tiles 128); CUDA cores otherwise
+  if (bsa::attend_tc_supported(*s) && W <= 1024 &&
+      (long long)s->B * s->Hq * s->N < (1ll << 31)) {
+    e = bsa::launch_attend_tc(*s, q, k, v, kv_idx, kv_cnt, W, scale, out, lse, dev_status, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "attend (tensor cores)");
+  } else {
+    e = bsa::launch_attend_simt(*s, q, k, v, kv_idx, kv_cnt, W, scale, out, lse, dev_status, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "attend");
+  }
   return ok();
 }
 

@@ -1,0 +1,407 @@
+// Block-sparse causal attention on Blackwell tensor cores (tcgen05 + TMEM + TMA).
+//
+// O_i = sum over the keys j of the listed blocks with j <= i of
+// softmax(scale * q_i . k_j) v_j -- the sparse aggregation step of [UGS]
+// step 5 and [Stem] Implementação: only the blocks in kv_idx are streamed,
+// with an online softmax. Shapes: bf16, d = 128, key blocks of 64, query
+// tiles of 128.
+//
+// One CTA per (batch, query head, query tile); 192 threads in four roles:
+//   warp 0 (one thread)  TMA producer: the Q tile once, then K and V tiles of
+//                        128 keys = two listed blocks gathered into adjacent
+//                        shared-memory rows, two stages deep.
+//   warp 1 (one thread)  MMA issuer: S_j = Q K_j^T into one of two TMEM
+//                        buffers, then O += P_j V_j into the TMEM accumulator.
+//                        S_{j+1} is issued before PV_j so the tensor core
+//                        works while the softmax warps handle tile j.
+//   warps 2-5            softmax: each thread owns one query row (= TMEM lane):
+//                        reads its S row, applies the causal mask on the
+//                        diagonal tile, keeps a running max and sum, writes P_j
+//                        (bf16) into 128-byte-swizzled shared memory, and
+//                        rescales its O row in TMEM only when its running max
+//                        grew by more than 2^8 (exact: the final division uses
+//                        the same max). Epilogue: O / l -> bf16, optional lse.
+// Operand layouts (all 128-byte swizzled, as TMA writes them):
+//   Q, K: K-major [rows x 64 elements] halves; P: K-major (keys are K);
+//   V: MN-major (rows = keys, 64 contiguous head dims per 128-byte row).
+// The CTA-to-work mapping walks (batch, KV head) outermost and the query heads
+// of a group innermost, so CTAs running together gather from one KV head and
+// reuse its blocks through L2.
+// Every mbarrier wait is bounded (tc::mbar_wait); a timeout sets
+// BSA_DEV_TIMEOUT, the CTA unwinds, waits for its own copies and MMAs, and
+// frees its TMEM. Invalid kv_idx entries are dropped with BSA_DEV_BAD_INDEX.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace bsa {
+
+namespace {
+constexpr int BQ = 128;          // query rows per tile
+constexpr int BKB = 64;          // keys per listed block
+constexpr int HD = 128;          // head dim
+constexpr int NS = 2;            // K/V pipeline stages
+constexpr int kThreads = 192;
+constexpr int kMaxList = 1024;   // kv_idx entries staged per tile
+constexpr uint32_t kHalf = 16384;            // [128 rows x 128 bytes]
+constexpr uint32_t kTile = 2 * kHalf;        // 128 rows x 128 dims bf16
+constexpr uint32_t kBoxK = 8192;             // one 64-key block half
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;                // S buffers at columns 0 and 128
+constexpr uint32_t kColO = 256;              // O accumulator
+
+struct __align__(8) Ctrl {
+  uint64_t q_full;
+  uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, o_ready, done;
+  uint32_t tmem;
+  int abort_flag;
+  int n_list;
+  int list[kMaxList];
+};
+
+constexpr size_t kSmemQ = 0;
+constexpr size_t kSmemK = kSmemQ + kTile;
+constexpr size_t kSmemV = kSmemK + NS * kTile;
+constexpr size_t kSmemP = kSmemV + NS * kTile;
+constexpr size_t kSmemCtrl = kSmemP + kTile;
+constexpr size_t kSmemBytes = kSmemCtrl + sizeof(Ctrl) + 1024;   // + alignment slack
+
+__device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
+    const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+    const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ kv_idx,
+    const int32_t* __restrict__ kv_cnt, int W, float scale_log2, uint16_t* __restrict__ out,
+    float* __restrict__ lse, int32_t* dev_status, int N, int Hq, int Hkv, int n_qt, int n_kb) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl& c = *reinterpret_cast<Ctrl*>(sm + kSmemCtrl);
+  const uint32_t sQ = tc::smem_u32(sm + kSmemQ);
+  const uint32_t sK = tc::smem_u32(sm + kSmemK);
+  const uint32_t sV = tc::smem_u32(sm + kSmemV);
+  const uint32_t sP = tc::smem_u32(sm + kSmemP);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = Hq / Hkv;
+  int x = blockIdx.x;
+  const int hh = x % G;
+  x /= G;
+  const int t = n_qt - 1 - (x % n_qt);
+  const int bgi = x / n_qt;                 // b * Hkv + g
+  const int b = bgi / Hkv, g = bgi % Hkv;
+  const int h = g * G + hh;
+  const size_t bh = (size_t)b * Hq + h;
+  const size_t krow = bh * n_qt + t;
+  const int J = ((t + 1) * BQ - 1) / BKB;   // last visible block
+  const int q_row0 = (int)(bh * N + (size_t)t * BQ);
+  const int kv_row0 = bgi * N;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&c.q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      tc::mbar_init(&c.k_full[s], 1);
+      tc::mbar_init(&c.k_empty[s], 1);
+      tc::mbar_init(&c.v_full[s], 1);
+      tc::mbar_init(&c.v_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&c.s_full[i], 1);
+      tc::mbar_init(&c.s_free[i], 4);
+    }
+    tc::mbar_init(&c.p_full, 4);
+    tc::mbar_init(&c.o_ready, 1);
+    tc::mbar_init(&c.done, 1);
+    c.abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&c.tmem, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (warp == 2) {
+    // compact the valid entries of this tile's kv_idx row into shared memory
+    int cnt = kv_cnt[krow];
+    if (cnt < 0 || cnt > W) {
+      if (lane == 0) set_status(dev_status, BSA_DEV_BAD_INDEX);
+      cnt = cnt < 0 ? 0 : W;
+    }
+    int n = 0;
+    for (int base = 0; base < cnt; base += 32) {
+      const int i = base + lane;
+      const int j = i < cnt ? kv_idx[krow * W + i] : -1;
+      const bool valid = i < cnt && j >= 0 && j < n_kb && j <= J;
+      const unsigned m = __ballot_sync(0xffffffffu, valid);
+      if (__any_sync(0xffffffffu, i < cnt && !valid) && lane == 0) set_status(dev_status, BSA_DEV_BAD_INDEX);
+      if (valid) c.list[n + __popc(m & ((1u << lane) - 1u))] = j;
+      n += __popc(m);
+    }
+    if (lane == 0) c.n_list = n;
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = c.tmem;
+  const int nl = c.n_list;
+  const int ntiles = (nl + 1) / 2;
+  volatile int* abort_flag = &c.abort_flag;
+  int k_issued = 0, v_issued = 0;     // tiles whose K / V loads the producer issued
+  bool mma_issued = false;
+
+  if (warp == 0 && lane == 0 && ntiles > 0) {
+    // ---------------- TMA producer ----------------
+    tc::prefetch_tmap(&tmq);
+    tc::prefetch_tmap(&tmk);
+    tc::prefetch_tmap(&tmv);
+    tc::mbar_arrive_expect_tx(&c.q_full, kTile);
+    tc::tma_load_2d(sm + kSmemQ, &tmq, 0, q_row0, &c.q_full);
+    tc::tma_load_2d(sm + kSmemQ + kHalf, &tmq, 64, q_row0, &c.q_full);
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % NS;
+      const int ja = c.list[2 * j];
+      const int jb = (2 * j + 1 < nl) ? c.list[2 * j + 1] : ja;
+      const int ra = kv_row0 + ja * BKB, rb = kv_row0 + jb * BKB;
+      if (j >= NS && !tc::mbar_wait(&c.k_empty[s], ((j / NS) - 1) & 1, abort_flag, dev_status)) break;
+      uint8_t* kd = sm + kSmemK + s * kTile;
+      tc::mbar_arrive_expect_tx(&c.k_full[s], kTile);
+      tc::tma_load_2d(kd, &tmk, 0, ra, &c.k_full[s]);
+      tc::tma_load_2d(kd + kBoxK, &tmk, 0, rb, &c.k_full[s]);
+      tc::tma_load_2d(kd + kHalf, &tmk, 64, ra, &c.k_full[s]);
+      tc::tma_load_2d(kd + kHalf + kBoxK, &tmk, 64, rb, &c.k_full[s]);
+      k_issued = j + 1;
+      if (j >= NS && !tc::mbar_wait(&c.v_empty[s], ((j / NS) - 1) & 1, abort_flag, dev_status)) break;
+      uint8_t* vd = sm + kSmemV + s * kTile;
+      tc::mbar_arrive_expect_tx(&c.v_full[s], kTile);
+      tc::tma_load_2d(vd, &tmv, 0, ra, &c.v_full[s]);
+      tc::tma_load_2d(vd + kBoxK, &tmv, 0, rb, &c.v_full[s]);
+      tc::tma_load_2d(vd + kHalf, &tmv, 64, ra, &c.v_full[s]);
+      tc::tma_load_2d(vd + kHalf + kBoxK, &tmv, 64, rb, &c.v_full[s]);
+      v_issued = j + 1;
+    }
+  } else if (warp == 1 && lane == 0 && ntiles > 0) {
+    // ---------------- MMA issuer ----------------
+    constexpr uint32_t idS = tc::idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t idPV = tc::idesc_bf16_f32(128, 128, false, true);
+    auto issue_s = [&](int j) {
+      const uint32_t kb = sK + (j % NS) * kTile;
+      const uint32_t d = tmem + kColS + (j % 2) * 128;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+        tc::umma_bf16(d, tc::sdesc_sw128(sQ + off, 16, 1024), tc::sdesc_sw128(kb + off, 16, 1024), idS,
+                      kk > 0);
+      }
+      tc::umma_commit(&c.s_full[j % 2]);
+      tc::umma_commit(&c.k_empty[j % NS]);
+    };
+    bool ok = tc::mbar_wait(&c.q_full, 0, abort_flag, dev_status) &&
+              tc::mbar_wait(&c.k_full[0], 0, abort_flag, dev_status);
+    if (ok) {
+      tc::tc_fence_after();
+      issue_s(0);
+      mma_issued = true;
+    }
+    for (int j = 0; ok && j < ntiles; ++j) {
+      const int jn = j + 1;
+      if (jn < ntiles) {
+        ok = tc::mbar_wait(&c.k_full[jn % NS], (jn / NS) & 1, abort_flag, dev_status) &&
+             (jn < 2 || tc::mbar_wait(&c.s_free[jn % 2], ((jn / 2) - 1) & 1, abort_flag, dev_status));
+        if (!ok) break;
+        tc::tc_fence_after();
+        issue_s(jn);
+      }
+      ok = tc::mbar_wait(&c.p_full, j & 1, abort_flag, dev_status) &&
+           tc::mbar_wait(&c.v_full[j % NS], (j / NS) & 1, abort_flag, dev_status);
+      if (!ok) break;
+      tc::tc_fence_after();
+      const uint32_t vb = sV + (j % NS) * kTile;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t aoff = (kk >> 2) * kHalf + (kk & 3) * 32;
+        tc::umma_bf16(tmem + kColO, tc::sdesc_sw128(sP + aoff, 16, 1024),
+                      tc::sdesc_sw128(vb + kk * 2048, kHalf, 1024), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      tc::umma_commit(&c.o_ready);
+      tc::umma_commit(&c.v_empty[j % NS]);
+    }
+  } else if (warp >= 2) {
+    // ---------------- softmax warps ----------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                  // row in the tile == TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int row_abs = t * BQ + r;
+    float m_used = -INFINITY;                           // running max, scaled log2 units
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      ok = warp_all(tc::mbar_wait(&c.s_full[j % 2], (j / 2) & 1, abort_flag, dev_status));
+      if (!ok) break;
+      tc::tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tc::tmem_ld32(tl + kColS + (j % 2) * 128 + cc * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(v[i]);
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&c.s_free[j % 2]);
+
+      const int ja = c.list[2 * j];
+      const bool has_b = 2 * j + 1 < nl;
+      const int jb = has_b ? c.list[2 * j + 1] : ja;
+      // keys of block ja are ja*64 .. ja*64+63; mask any key after this row
+      const bool diag = (ja * BKB + BKB - 1 > t * BQ) || (jb * BKB + BKB - 1 > t * BQ) || !has_b;
+      float mx = -INFINITY;
+      if (diag) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const int key = (i < 64 ? ja : jb) * BKB + (i & 63);
+          const bool vis = key <= row_abs && (i < 64 || has_b);
+          s[i] = vis ? s[i] : -INFINITY;
+          mx = fmaxf(mx, s[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      }
+      const float m_tile = mx * scale_log2;
+      float alpha = 1.f;
+      if (m_tile > m_used + 8.0f) {                     // also taken when m_used is -inf
+        alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - m_tile);
+        m_used = m_tile;
+      }
+      const float m_safe = (m_used == -INFINITY) ? 0.f : m_used;
+      float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 128; i += 4) {
+        const float p0 = exp2f(fmaf(s[i], scale_log2, -m_safe));
+        const float p1 = exp2f(fmaf(s[i + 1], scale_log2, -m_safe));
+        const float p2 = exp2f(fmaf(s[i + 2], scale_log2, -m_safe));
+        const float p3 = exp2f(fmaf(s[i + 3], scale_log2, -m_safe));
+        sum0 += p0; sum1 += p1; sum2 += p2; sum3 += p3;
+        __nv_bfloat162 a = __floats2bfloat162_rn(p0, p1);
+        __nv_bfloat162 bq = __floats2bfloat162_rn(p2, p3);
+        pk[i / 2] = *reinterpret_cast<uint32_t*>(&a);
+        pk[i / 2 + 1] = *reinterpret_cast<uint32_t*>(&bq);
+      }
+      l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
+
+      if (j > 0) {
+        ok = warp_all(tc::mbar_wait(&c.o_ready, (j - 1) & 1, abort_flag, dev_status));
+        if (!ok) break;
+        tc::tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t v[32];
+            tc::tmem_ld32(tl + kColO + cc * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+            tc::tmem_st32(tl + kColO + cc * 32, v);
+          }
+        }
+      }
+      // P row -> shared memory, 128-byte swizzle: 16-byte chunk cc of row r at cc ^ (r & 7)
+      uint8_t* prow = sm + kSmemP + r * 128;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const int w0 = half * 32 + cc * 4;
+          uint4 v4 = make_uint4(pk[w0], pk[w0 + 1], pk[w0 + 2], pk[w0 + 3]);
+          *reinterpret_cast<uint4*>(prow + half * kHalf + ((cc ^ (r & 7)) * 16)) = v4;
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&c.p_full);
+    }
+    // epilogue
+    uint16_t* orow = out + ((size_t)bh * N + (size_t)t * BQ + r) * HD;
+    bool have = ok && ntiles > 0;
+    if (have) have = warp_all(tc::mbar_wait(&c.o_ready, (ntiles - 1) & 1, abort_flag, dev_status));
+    if (have) {
+      tc::tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tc::tmem_ld32(tl + kColO + cc * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 p = __floats2bfloat162_rn(__uint_as_float(v[i + 2 * e]) * inv,
+                                                     __uint_as_float(v[i + 2 * e + 1]) * inv);
+            w[e] = *reinterpret_cast<uint32_t*>(&p);
+          }
+          *reinterpret_cast<uint4*>(orow + cc * 32 + i) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      if (lse) lse[bh * N + (size_t)t * BQ + r] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    } else if (ntiles == 0) {
+#pragma unroll
+      for (int i = 0; i < HD; i += 8)
+        *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
+      if (lse) lse[bh * N + (size_t)t * BQ + r] = -INFINITY;
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0 && lane == 0 && ntiles > 0) {
+    // make sure no TMA copy of this CTA is still landing in shared memory: wait for
+    // the last phase issued on every stage (earlier phases completed before it)
+    for (int j = k_issued - NS < 0 ? 0 : k_issued - NS; j < k_issued; ++j)
+      tc::mbar_wait_timed(&c.k_full[j % NS], (j / NS) & 1);
+    for (int j = v_issued - NS < 0 ? 0 : v_issued - NS; j < v_issued; ++j)
+      tc::mbar_wait_timed(&c.v_full[j % NS], (j / NS) & 1);
+  }
+  if (warp == 1) {
+    if (lane == 0 && mma_issued) {
+      // every MMA this thread issued has completed once this commit arrives
+      tc::umma_commit(&c.done);
+      tc::mbar_wait_timed(&c.done, 0);
+    }
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+bool attend_tc_supported(const bsa_shape& s) {
+  return s.dtype == BSA_BF16 && s.d == HD && s.block_k == BKB && s.tile_q == BQ;
+}
+
+cudaError_t launch_attend_tc(const bsa_shape& s, const void* q, const void* k, const void* v,
+                             const int32_t* kv_idx, const int32_t* kv_cnt, int W, float scale,
+                             void* out, float* lse, int32_t* dev_status, cudaStream_t st) {
+  if (W > kMaxList) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv;
+  const uint64_t qrows = (uint64_t)s.B * s.Hq * s.N, krows = (uint64_t)s.B * s.Hkv * s.N;
+  if (!make_tmap_bf16_2d(&mq, q, qrows, HD, 64, BQ) || !make_tmap_bf16_2d(&mk, k, krows, HD, 64, BKB) ||
+      !make_tmap_bf16_2d(&mv, v, krows, HD, 64, BKB))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int n_qt = s.N / BQ;
+  const long long grid = (long long)s.B * s.Hq * n_qt;
+  attend_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(
+      mq, mk, mv, kv_idx, kv_cnt, W, scale * 1.4426950408889634f, (uint16_t*)out, lse, dev_status,
+      s.N, s.Hq, s.Hkv, n_qt, s.N / BKB);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -293,15 +293,22 @@ def attend_tile(Q_tile: np.ndarray, K: np.ndarray, V: np.ndarray, kv_row: np.nda
     the softmax denominator."""
     Qt = widen(Q_tile)
     blocks = [int(j) for j in kv_row if j >= 0]
+    if not blocks:
+        return np.zeros((Qt.shape[0], K.shape[-1])), np.full(Qt.shape[0], -np.inf)
     keys = np.concatenate([np.arange(j * block_k, (j + 1) * block_k) for j in blocks])
     Kt, Vt = widen(K[keys]), widen(V[keys])
     logits = scale * (Qt @ Kt.T)
     rows = row0 + np.arange(Qt.shape[0])
     logits[keys[None, :] > rows[:, None]] = -np.inf
-    mx = logits.max(axis=1, keepdims=True)
+    seen = np.isfinite(logits).any(axis=1)
+    # a row that sees no key of the listed blocks (possible only for a caller-made
+    # list without the tile's own block) has an empty softmax: output 0, lse -inf
+    mx = np.where(seen, logits.max(axis=1), 0.0)[:, None]
     p = np.exp(logits - mx)
     den = p.sum(axis=1, keepdims=True)
-    return (p @ Vt) / den, (mx + np.log(den))[:, 0]
+    out = np.where(seen[:, None], (p @ Vt) / np.where(den > 0, den, 1.0), 0.0)
+    lse = np.where(seen, (mx + np.log(np.where(den > 0, den, 1.0)))[:, 0], -np.inf)
+    return out, lse
 
 
 def attend(Q, K, V, kv_idx, tile_q, block_k, scale, tiles=None):

@@ -201,3 +201,40 @@ def test_decode_shapes(Hq, Hkv, d, bkv):
     spec = S.DecodeSpec("dec", B=2, Hq=Hq, Hkv=Hkv, L=2048, d=d, block_kv=bkv, tau=1e-2,
                         phi=1e-3, patience=2)
     _check_decode(spec, 1012, spec.tau, spec.phi, spec.patience)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_attend_arbitrary_lists(dtype):
+    """Caller-made kv_idx rows: unsorted, odd and even counts, duplicates of
+    nothing, rows without their diagonal block (their early rows see no key:
+    output 0, lse -inf), and entries beyond kv_cnt that must be ignored."""
+    spec = S.PrefillSpec("lists", B=1, Hq=4, Hkv=2, N=2048, d=128, block_k=64, tile_q=128,
+                         k_first=8, k_last=8, rho=1, gate_quantile=0.25, score_kind="mean",
+                         dtype=dtype, structure="iid")
+    (q, k, v), (qd, kd, vd) = inputs(spec, 1013)
+    rng = np.random.default_rng(5)
+    n_qt, W = spec.n_qt, 9
+    kv = np.full((1, 4, n_qt, W), -1, np.int32)
+    cnt = np.zeros((1, 4, n_qt), np.int32)
+    for h in range(4):
+        for t in range(n_qt):
+            J = 2 * t + 1
+            c = int(rng.integers(0, min(W, J + 1) + 1))
+            sel = rng.permutation(J + 1)[:c]
+            kv[0, h, t, :c] = sel
+            kv[0, h, t, c:] = rng.integers(0, J + 1, size=W - c)   # ignored garbage
+            cnt[0, h, t] = c
+    kvd, cntd = torch.from_numpy(kv).cuda(), torch.from_numpy(cnt).cuda()
+    out, lse, st = bb.attend(qd, kd, vd, kvd, cntd, block_k=64, tile_q=128, want_lse=True)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    kv_used = kv.copy()
+    for h in range(4):
+        for t in range(n_qt):
+            kv_used[0, h, t, cnt[0, h, t]:] = -1
+    ro, rl = O.attend(q, k, v, kv_used, 128, 64, 1 / math.sqrt(128))
+    check_attend(out_rows(out), ro)
+    gl = lse.cpu().numpy()
+    assert np.array_equal(np.isneginf(gl), np.isneginf(rl))
+    fin = np.isfinite(rl)
+    np.testing.assert_allclose(gl[fin], rl[fin], atol=1e-3)

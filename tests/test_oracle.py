@@ -471,3 +471,22 @@ def test_generator_structure():
     a = S.prefill_head(spec, 5, "q", 0, 3)
     b = S.prefill_head(spec, 5, "q", 0, 3)
     assert np.array_equal(a, b)
+
+
+def test_attend_empty_rows():
+    """Rows that see no listed key (a caller-made list without the tile's own
+    block) get output 0 and lse -inf; rows that do see keys are unaffected."""
+    rng = np.random.default_rng(12)
+    N, d, tile_q, bk = 256, 8, 64, 64
+    Q = rng.standard_normal((N, d)).astype(np.float32)
+    K = rng.standard_normal((N, d)).astype(np.float32)
+    V = rng.standard_normal((N, d)).astype(np.float32)
+    # tile 1 (rows 64..127) lists only block 1: every row sees keys 64..row
+    o, l = O.attend_tile(Q[64:128], K, V, np.array([1, -1]), 64, bk, 0.3)
+    assert np.isfinite(l).all()
+    # tile 0 listing nothing at all
+    o, l = O.attend_tile(Q[0:64], K, V, np.array([-1, -1]), 0, bk, 0.3)
+    assert (o == 0).all() and np.isneginf(l).all()
+    # tile 1 listing only block 2, which is after every row of the tile
+    o, l = O.attend_tile(Q[64:128], K, V, np.array([2]), 64, bk, 0.3)
+    assert (o == 0).all() and np.isneginf(l).all()
