@@ -261,6 +261,7 @@ def main_gpu(args):
     kv_cnt = torch.empty(B, Hq, n_qt, dtype=torch.int32, device=dev)
     out = torch.empty_like(q)
     st_sel = torch.zeros(1, dtype=torch.int32, device=dev)
+    st_score = torch.zeros(1, dtype=torch.int32, device=dev)
     st_att = torch.zeros(1, dtype=torch.int32, device=dev)
     theta = torch.empty(1, dtype=torch.float32, device=dev)
     ws_s_n = bb.bsa_score_workspace_bytes(shape, bb.BSA_SCORE_MEAN)
@@ -273,7 +274,7 @@ def main_gpu(args):
     def step(q_, k_, v_, out_, ev=None):
         if ev:
             ev[0].record(stream)
-        bb.bsa_score(shape, bb.BSA_SCORE_MEAN, q_, k_, None, scores, ws_s, ws_s_n, sh)
+        bb.bsa_score(shape, bb.BSA_SCORE_MEAN, q_, k_, None, scores, st_score, ws_s, ws_s_n, sh)
         if ev:
             ev[1].record(stream)
         bb.bsa_select(shape, prm, scores, kv_idx, kv_cnt, None, None, None, theta, st_sel,
@@ -287,7 +288,7 @@ def main_gpu(args):
     for _ in range(args.warmup):
         step(q, k, v, out)
     torch.cuda.synchronize()
-    assert int(st_sel.item()) == 0 and int(st_att.item()) == 0
+    assert int(st_sel.item()) == 0 and int(st_att.item()) == 0 and int(st_score.item()) == 0
     sel_blocks = int(kv_cnt.sum().item())
     flops = 4.0 * spec.tile_q * spec.block_k * d * sel_blocks
     # unmasked (i, j) pairs of the selected blocks, for the alternative count

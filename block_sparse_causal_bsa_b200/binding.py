@@ -77,7 +77,7 @@ def lib() -> ctypes.CDLL:
         dsp, dpp = ctypes.POINTER(DecodeShape), ctypes.POINTER(DecodeParams)
         L.bsa_score_workspace_bytes.argtypes = [sp, ctypes.c_int]
         L.bsa_score_workspace_bytes.restype = sz
-        L.bsa_score.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, vp, sz, vp]
+        L.bsa_score.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, i32p, vp, sz, vp]
         L.bsa_score.restype = ctypes.c_int
         L.bsa_kv_idx_width.argtypes = [sp, pp]
         L.bsa_kv_idx_width.restype = ctypes.c_int
@@ -157,9 +157,9 @@ def bsa_score_workspace_bytes(shape: Shape, kind: int) -> int:
     return lib().bsa_score_workspace_bytes(ctypes.byref(shape), kind)
 
 
-def bsa_score(shape, kind, q, k, v, scores, ws, ws_bytes, stream=None) -> None:
+def bsa_score(shape, kind, q, k, v, scores, dev_status, ws, ws_bytes, stream=None) -> None:
     _check(lib().bsa_score(ctypes.byref(shape), kind, _ptr(q), _ptr(k), _ptr(v), _ptr(scores),
-                           _ptr(ws), ws_bytes, _stream(stream)))
+                           _ptr(dev_status), _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def bsa_kv_idx_width(shape: Shape, params: SelectParams) -> int:
@@ -206,14 +206,15 @@ def _empty_bytes(n: int, device) -> torch.Tensor:
     return torch.empty(max(int(n), 256), dtype=torch.uint8, device=device)
 
 
-def score(q, k, v=None, *, block_k: int, tile_q: int, output_aware: bool = False, stream=None):
+def score(q, k, v=None, *, block_k: int, tile_q: int, output_aware: bool = False, stream=None,
+          status: Optional[torch.Tensor] = None):
     shape = make_shape(q, k, block_k, tile_q)
     kind = BSA_SCORE_MEAN_VNORM if output_aware else BSA_SCORE_MEAN
     B, Hq, N, _ = q.shape
     scores = torch.empty(B, Hq, N // tile_q, N // block_k, dtype=torch.float32, device=q.device)
     nb = bsa_score_workspace_bytes(shape, kind)
     ws = _empty_bytes(nb, q.device)
-    bsa_score(shape, kind, q, k, v if output_aware else None, scores, ws, nb, stream)
+    bsa_score(shape, kind, q, k, v if output_aware else None, scores, status, ws, nb, stream)
     return scores
 
 
@@ -273,8 +274,11 @@ def prefill(q, k, v, *, block_k: int, tile_q: int, cfg: SelectConfig, output_awa
             scale: Optional[float] = None, stream=None):
     """score -> select -> attend on the current stream; returns (out, selection dict, status)."""
     shape = make_shape(q, k, block_k, tile_q)
-    s = score(q, k, v, block_k=block_k, tile_q=tile_q, output_aware=output_aware, stream=stream)
+    st_score = torch.zeros(1, dtype=torch.int32, device=q.device)
+    s = score(q, k, v, block_k=block_k, tile_q=tile_q, output_aware=output_aware, stream=stream,
+              status=st_score)
     sel = select(s, shape=shape, cfg=cfg, stream=stream)
+    sel["score_status"] = st_score
     out, _, st = attend(q, k, v, sel["kv_idx"], sel["kv_cnt"], block_k=block_k, tile_q=tile_q,
                         scale=scale, stream=stream)
     sel["scores"] = s

@@ -138,7 +138,8 @@ size_t bsa_score_workspace_bytes(const bsa_shape* s, bsa_score_kind kind) {
 }
 
 bsa_status bsa_score(const bsa_shape* s, bsa_score_kind kind, const void* q, const void* k,
-                     const void* v, float* scores, void* ws, size_t ws_bytes, void* stream) {
+                     const void* v, float* scores, int32_t* dev_status, void* ws, size_t ws_bytes,
+                     void* stream) {
   bsa_status st = check_shape(s);
   if (st != BSA_OK) return st;
   if (kind != BSA_SCORE_MEAN && kind != BSA_SCORE_MEAN_VNORM)
@@ -150,11 +151,22 @@ bsa_status bsa_score(const bsa_shape* s, bsa_score_kind kind, const void* q, con
   ScoreWs w = score_ws(*s, kind, ws);
   if (ws_bytes < w.bytes) return fail(BSA_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, w.bytes);
   cudaStream_t cs = (cudaStream_t)stream;
-  cudaError_t e = bsa::launch_pool(*s, k, kind == BSA_SCORE_MEAN_VNORM ? v : nullptr, w.kbar,
-                                   s->dtype == BSA_BF16 ? w.hi : nullptr, w.lo, w.w, cs);
+  cudaError_t e;
+  if (dev_status) {
+    e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
+  }
+  e = bsa::launch_pool(*s, k, kind == BSA_SCORE_MEAN_VNORM ? v : nullptr, w.kbar,
+                       s->dtype == BSA_BF16 ? w.hi : nullptr, w.lo, w.w, cs);
   if (e != cudaSuccess) return cuda_fail(e, "pool");
-  e = bsa::launch_score_simt(*s, q, w.kbar, w.w, scores, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "score");
+  // tensor-core path for bf16, d 128, query tiles of 128; CUDA cores otherwise
+  if (bsa::score_tc_supported(*s)) {
+    e = bsa::launch_score_tc(*s, q, w.hi, w.lo, w.w, scores, dev_status, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "score (tensor cores)");
+  } else {
+    e = bsa::launch_score_simt(*s, q, w.kbar, w.w, scores, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "score");
+  }
   return ok();
 }
 

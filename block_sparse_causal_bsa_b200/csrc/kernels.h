@@ -18,6 +18,7 @@ cudaError_t launch_score_simt(const bsa_shape& s, const void* q, const float* kb
                               const float* wnorm, float* scores, cudaStream_t st);
 
 // Block scores on tcgen05 tensor cores (bf16 inputs, hi/lo split of the pooled keys).
+bool score_tc_supported(const bsa_shape& s);
 cudaError_t launch_score_tc(const bsa_shape& s, const void* q, const uint16_t* kbar_hi,
                             const uint16_t* kbar_lo, const float* wnorm, float* scores,
                             int32_t* dev_status, cudaStream_t st);

@@ -134,10 +134,12 @@ size_t bsa_score_workspace_bytes(const bsa_shape* shape, bsa_score_kind kind);
 /* scores [B,Hq,n_qt,n_kb] fp32: s(t,j) for j <= J_t, -inf for j > J_t.
  * No 1/sqrt(d) factor (a common positive factor changes neither the ranking nor sigma).
  * The tile max runs over all tile_q rows, unmasked.
- * q, k: inputs of `shape->dtype`; v is read only for BSA_SCORE_MEAN_VNORM (else may be NULL). */
+ * q, k: inputs of `shape->dtype`; v is read only for BSA_SCORE_MEAN_VNORM (else may be NULL).
+ * dev_status: device int32 or NULL (BSA_DEV_TIMEOUT if a bounded wait ran out). */
 bsa_status bsa_score(const bsa_shape* shape, bsa_score_kind kind,
                      const void* q, const void* k, const void* v,
-                     float* scores, void* workspace, size_t workspace_bytes, void* stream);
+                     float* scores, int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                     void* stream);
 
 /* ---- selection ([UGS] steps 2-5; [Stem] 2.A) -------------------------------------- */
 

@@ -70,7 +70,7 @@ def test_workspace_sizes():
 def test_bad_shapes_rejected(bad):
     s = _shape(**bad)
     L = bb.lib()
-    st = L.bsa_score(ctypes.byref(s), 0, 16, 16, None, 16, 256, 1 << 30, None)
+    st = L.bsa_score(ctypes.byref(s), 0, 16, 16, None, 16, None, 256, 1 << 30, None)
     assert st in (bb.BSA_ERR_INVALID_ARG, bb.BSA_ERR_UNSUPPORTED)
     assert L.bsa_last_error()
     p = bb.SelectParams(8, 8, 1, 0.25, 0.0)
@@ -81,14 +81,14 @@ def test_bad_shapes_rejected(bad):
 def test_null_pointers_rejected():
     L = bb.lib()
     s = _shape()
-    assert L.bsa_score(ctypes.byref(s), 0, None, 16, None, 16, 256, 1 << 30, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_score(ctypes.byref(s), 0, None, 16, None, 16, None, 256, 1 << 30, None) == bb.BSA_ERR_INVALID_ARG
     # output-aware score without V
-    assert L.bsa_score(ctypes.byref(s), 1, 16, 16, None, 16, 256, 1 << 30, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_score(ctypes.byref(s), 1, 16, 16, None, 16, None, 256, 1 << 30, None) == bb.BSA_ERR_INVALID_ARG
     # undersized workspace
-    assert L.bsa_score(ctypes.byref(s), 0, 16, 16, None, 16, 256, 10, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_score(ctypes.byref(s), 0, 16, 16, None, 16, None, 256, 10, None) == bb.BSA_ERR_INVALID_ARG
     assert b"workspace" in L.bsa_last_error()
     # misaligned pointer
-    assert L.bsa_score(ctypes.byref(s), 0, 18, 16, None, 16, 256, 1 << 30, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_score(ctypes.byref(s), 0, 18, 16, None, 16, None, 256, 1 << 30, None) == bb.BSA_ERR_INVALID_ARG
     assert L.bsa_attend(ctypes.byref(s), 16, 16, 16, 16, 16, 128, 0.1, 16, None, None, None) == bb.BSA_ERR_INVALID_ARG
     assert L.bsa_attend(ctypes.byref(s), 16, 16, 16, 16, 16, 0, 0.1, 16, None, 16, None) == bb.BSA_ERR_INVALID_ARG
     assert L.bsa_attend(ctypes.byref(s), 16, 16, 16, 16, 16, 128, -1.0, 16, None, 16, None) == bb.BSA_ERR_INVALID_ARG

@@ -1,0 +1,118 @@
+"""Full-size parity: every workload at its real size, through the same C-ABI
+calls the benchmark times. Outputs the oracle cannot afford in full are
+sampled: block-score rows and attention tiles (first, last, triggered and
+seeded random ones); the selection is compared bit for bit over the whole
+layer (the oracle ranks every row of the GPU's own scores); decode replays the
+termination rule on every group's probe trace and runs the oracle end to end
+on a sample of groups."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_causal_bsa_b200 import binding as bb
+from block_sparse_causal_bsa_b200 import synthetic as S
+from oracle import bsa_oracle as O
+
+from gpu_util import check_attend, check_scores, check_selection, out_rows, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_prefill(name, seed, n_rows=24, n_tiles=12):
+    spec = S.WORKLOADS[name]
+    q, k, v = S.prefill_inputs(spec, seed)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    oam = spec.score_kind == "mean_vnorm"
+    cfg = bb.SelectConfig(spec.k_first, spec.k_last, spec.rho, spec.gate_quantile)
+    out, sel, st = bb.prefill(qd, kd, vd, block_k=spec.block_k, tile_q=spec.tile_q, cfg=cfg,
+                              output_aware=oam)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and int(sel["dev_status"].item()) == 0
+    assert int(sel["score_status"].item()) == 0
+    G = spec.Hq // spec.Hkv
+    rng = np.random.default_rng(seed)
+    gs = sel["scores"].cpu().numpy()
+    # block scores: sampled rows, oracle pooling of the KV heads they need
+    rows = [(int(rng.integers(spec.B)), int(rng.integers(spec.Hq)), int(rng.integers(spec.n_qt)))
+            for _ in range(n_rows)] + [(0, 0, 0), (spec.B - 1, spec.Hq - 1, spec.n_qt - 1)]
+    kbar, wn = {}, {}
+    for b, h, t in rows:
+        g = h // G
+        if (b, g) not in kbar:
+            kbar[b, g] = O.pool_keys(k[b, g], spec.block_k)
+            wn[b, g] = O.value_block_norm(v[b, g], spec.block_k) if oam else None
+        _, J = O.tile_blocks(t, spec.tile_q, spec.block_k)
+        ref = O.score_tile(q[b, h, t * spec.tile_q:(t + 1) * spec.tile_q], kbar[b, g], J, wn[b, g])
+        check_scores(gs[b, h, t][None], ref[None])
+    # selection: the whole layer, bit for bit on the GPU's scores
+    ref_sel = O.select(gs, spec.tile_q, spec.block_k, spec.k_first, spec.k_last, spec.rho,
+                       spec.gate_quantile)
+    check_selection(sel, ref_sel)
+    # attend: sampled tiles, including the first, the last and triggered ones
+    tiles = [(0, 0, 0), (spec.B - 1, spec.Hq - 1, spec.n_qt - 1)]
+    trig = np.argwhere(ref_sel["trigger"] > 0)
+    for b, t in trig[rng.permutation(len(trig))[:3]]:
+        tiles.append((int(b), int(rng.integers(spec.Hq)), int(t)))
+    tiles += [(int(rng.integers(spec.B)), int(rng.integers(spec.Hq)), int(rng.integers(spec.n_qt)))
+              for _ in range(n_tiles)]
+    go = out_rows(out)
+    scale = 1.0 / math.sqrt(spec.d)
+    for b, h, t in tiles:
+        r0 = t * spec.tile_q
+        ro, _ = O.attend_tile(q[b, h, r0:r0 + spec.tile_q], k[b, h // G], v[b, h // G],
+                              ref_sel["kv_idx"][b, h, t], r0, spec.block_k, scale)
+        check_attend(go[b, h, r0:r0 + spec.tile_q], ro)
+    return spec, ref_sel
+
+
+def test_full_prefill_32k_vs():
+    _full_prefill("prefill_32k_vs", 1002)
+
+
+def test_full_gated_prefill_128k():
+    spec, r = _full_prefill("gated_prefill_128k", 1003)
+    cut_tiles = int(r["cut"].sum()) * spec.B
+    ntrig = int(r["trigger"].sum())
+    # a quantile gate at q = 0.25 fires on about a quarter of the cut tiles
+    assert 0.15 * cut_tiles <= ntrig <= 0.3 * cut_tiles
+    assert r["kv_cnt"].max() <= r["W"] == 128
+
+
+def test_full_tpd_oam_prefill_64k():
+    spec, r = _full_prefill("tpd_oam_prefill_64k", 1004)
+    # position-decay budget: the first tiles keep more blocks than the last
+    cnt = r["kv_cnt"]
+    assert cnt[:, :, 100].max() > cnt[:, :, -1].max()
+    assert cnt[:, :, -1].max() == 32 + 0 and cnt[:, :, 64].min() == 128 - (96 * 64) // 511
+
+
+def test_full_decode_art_64k():
+    spec = S.DECODE_WORKLOADS["decode_art_64k"]
+    q, k, v = S.decode_inputs(spec, 1005)
+    dims = S.default_probe_dims(32)
+    out, used, trace, st = bb.decode(to_dev(q), to_dev(k), to_dev(v), block_kv=spec.block_kv,
+                                     tau=spec.tau, phi=spec.phi, patience=spec.patience,
+                                     probe_dims=dims, want_trace=True)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    used, trace, go = used.cpu().numpy(), trace.cpu().numpy(), out_rows(out)
+    nb = spec.L // spec.block_kv
+    G = spec.Hq // spec.Hkv
+    for b in range(spec.B):
+        for g in range(spec.Hkv):
+            assert used[b, g] == O.termination_block(trace[b, g], spec.tau, spec.phi, spec.patience,
+                                                     n_blocks=nb)
+    rng = np.random.default_rng(5)
+    agree = 0
+    sample = [(int(rng.integers(spec.B)), int(rng.integers(spec.Hkv))) for _ in range(8)]
+    for b, g in sample:
+        u = int(used[b, g])
+        o_ref, _, _ = O.decode_group(q[b, g * G:(g + 1) * G], k[b, g, :u * 128], v[b, g, :u * 128], 128,
+                                     1 / math.sqrt(128), spec.tau, spec.phi, 1, dims, enable=False)
+        check_attend(go[b, g * G:(g + 1) * G], o_ref)
+        _, u_ref, _ = O.decode_group(q[b, g * G:(g + 1) * G], k[b, g], v[b, g], 128,
+                                     1 / math.sqrt(128), spec.tau, spec.phi, 1, dims)
+        agree += int(u_ref == u)
+    assert agree >= 6

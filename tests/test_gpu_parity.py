@@ -35,6 +35,7 @@ def _run_prefill(spec, seed, k_first=None, k_last=None, tiles=None):
                               output_aware=oam)
     torch.cuda.synchronize()
     assert int(st.item()) == 0 and int(sel["dev_status"].item()) == 0
+    assert int(sel["score_status"].item()) == 0
     g_scores = sel["scores"].cpu().numpy()
     ref_scores = O.block_scores(q, k, spec.tile_q, spec.block_k, V=v if oam else None)
     check_scores(g_scores, ref_scores)
