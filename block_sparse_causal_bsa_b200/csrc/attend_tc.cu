@@ -6,7 +6,7 @@
 // with an online softmax. Shapes: bf16, d = 128, key blocks of 64, query
 // tiles of 128.
 //
-// One CTA per (batch, query head, query tile); 192 threads in four roles:
+// One CTA per (batch, query head, query tile); 320 threads in four roles:
 //   warp 0 (one thread)  TMA producer: the Q tile once, then K and V tiles of
 //                        128 keys = two listed blocks gathered into adjacent
 //                        shared-memory rows, two stages deep.
@@ -14,11 +14,15 @@
 //                        buffers, then O += P_j V_j into the TMEM accumulator.
 //                        S_{j+1} is issued before PV_j so the tensor core
 //                        works while the softmax warps handle tile j.
-//   warps 2-5            softmax: each thread owns one query row (= TMEM lane):
-//                        reads its S row, applies the causal mask on the
-//                        diagonal tile, keeps a running max and sum, writes P_j
-//                        (bf16) into 128-byte-swizzled shared memory, and
-//                        rescales its O row in TMEM only when its running max
+//   warps 2-9            softmax: two warps per TMEM lane quarter; a thread owns
+//                        half of one query row (64 of the tile's 128 keys, i.e.
+//                        one listed block). The two halves of a row exchange
+//                        their tile max through shared memory (a 64-thread
+//                        named barrier per lane quarter), then each applies the
+//                        causal mask on the diagonal tile, exponentiates, keeps
+//                        its part of the row sum, writes its half of P_j (bf16)
+//                        into 128-byte-swizzled shared memory, and rescales its
+//                        half of the O row in TMEM only when the running max
 //                        grew by more than 2^8 (exact: the final division uses
 //                        the same max). Epilogue: O / l -> bf16, optional lse.
 // Operand layouts (all 128-byte swizzled, as TMA writes them):
@@ -43,7 +47,8 @@ constexpr int BQ = 128;          // query rows per tile
 constexpr int BKB = 64;          // keys per listed block
 constexpr int HD = 128;          // head dim
 constexpr int NS = 2;            // K/V pipeline stages
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxWarps = 8;
 constexpr int kMaxList = 1024;   // kv_idx entries staged per tile
 constexpr uint32_t kHalf = 16384;            // [128 rows x 128 bytes]
 constexpr uint32_t kTile = 2 * kHalf;        // 128 rows x 128 dims bf16
@@ -60,6 +65,10 @@ struct __align__(8) Ctrl {
   uint32_t tmem;
   int abort_flag;
   int n_list;
+  uint64_t xbar[4];          // per lane quarter: both half-row maxima written (one phase per tile)
+  uint64_t lbar[4];          // per lane quarter: both row-sum parts written (once)
+  float xmax[2][2][128];     // [tile parity][half][row] max of the half-row
+  float lpart[2][128];       // [half][row] row-sum part
   int list[kMaxList];
 };
 
@@ -71,6 +80,12 @@ constexpr size_t kSmemCtrl = kSmemP + kTile;
 constexpr size_t kSmemBytes = kSmemCtrl + sizeof(Ctrl) + 1024;   // + alignment slack
 
 __device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
@@ -111,9 +126,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&c.s_full[i], 1);
-      tc::mbar_init(&c.s_free[i], 4);
+      tc::mbar_init(&c.s_free[i], kSoftmaxWarps);
     }
-    tc::mbar_init(&c.p_full, 4);
+    tc::mbar_init(&c.p_full, kSoftmaxWarps);
+    for (int q = 0; q < 4; ++q) {
+      tc::mbar_init(&c.xbar[q], 2);
+      tc::mbar_init(&c.lbar[q], 2);
+    }
     tc::mbar_init(&c.o_ready, 1);
     tc::mbar_init(&c.done, 1);
     c.abort_flag = 0;
@@ -231,21 +250,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
   } else if (warp >= 2) {
     // ---------------- softmax warps ----------------
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;                   // 0: keys 0-63 of the tile, 1: keys 64-127
     const int r = quarter * 32 + lane;                  // row in the tile == TMEM lane
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const int row_abs = t * BQ + r;
     float m_used = -INFINITY;                           // running max, scaled log2 units
-    float l = 0.f;
+    float l = 0.f;                                      // this half's part of the row sum
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       ok = warp_all(tc::mbar_wait(&c.s_full[j % 2], (j / 2) & 1, abort_flag, dev_status));
       if (!ok) break;
       tc::tc_fence_after();
-      float s[128];
+      float s[64];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32];
-        tc::tmem_ld32(tl + kColS + (j % 2) * 128 + cc * 32, v);
+        tc::tmem_ld32(tl + kColS + (j % 2) * 128 + half * 64 + cc * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(v[i]);
       }
@@ -253,39 +273,49 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c.s_free[j % 2]);
 
-      const int ja = c.list[2 * j];
       const bool has_b = 2 * j + 1 < nl;
-      const int jb = has_b ? c.list[2 * j + 1] : ja;
-      // keys of block ja are ja*64 .. ja*64+63; mask any key after this row
-      const bool diag = (ja * BKB + BKB - 1 > t * BQ) || (jb * BKB + BKB - 1 > t * BQ) || !has_b;
-      float mx = -INFINITY;
+      const int blk = half == 0 ? c.list[2 * j] : (has_b ? c.list[2 * j + 1] : -1);
+      // mask: keys after this row, and the empty second slot of an odd tail
+      const bool diag = blk < 0 || blk * BKB + BKB - 1 > t * BQ;
+      float mx8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
       if (diag) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const int key = (i < 64 ? ja : jb) * BKB + (i & 63);
-          const bool vis = key <= row_abs && (i < 64 || has_b);
+        for (int i = 0; i < 64; ++i) {
+          const bool vis = blk >= 0 && blk * BKB + i <= row_abs;
           s[i] = vis ? s[i] : -INFINITY;
-          mx = fmaxf(mx, s[i]);
+          mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, s[i]);
+        for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
       }
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      // share the half-row max with the partner warp (buffer alternates by tile parity;
+      // a buffer is rewritten two tiles later, after the partner passed the next exchange)
+      c.xmax[j & 1][half][r] = mx;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&c.xbar[quarter]);
+      ok = warp_all(tc::mbar_wait(&c.xbar[quarter], j & 1, abort_flag, dev_status));
+      if (!ok) break;
+      mx = fmaxf(mx, c.xmax[j & 1][half ^ 1][r]);
       const float m_tile = mx * scale_log2;
       float alpha = 1.f;
       if (m_tile > m_used + 8.0f) {                     // also taken when m_used is -inf
-        alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - m_tile);
+        alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_tile);
         m_used = m_tile;
       }
       const float m_safe = (m_used == -INFINITY) ? 0.f : m_used;
       float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
-      uint32_t pk[64];
+      uint32_t pk[32];
 #pragma unroll
-      for (int i = 0; i < 128; i += 4) {
-        const float p0 = exp2f(fmaf(s[i], scale_log2, -m_safe));
-        const float p1 = exp2f(fmaf(s[i + 1], scale_log2, -m_safe));
-        const float p2 = exp2f(fmaf(s[i + 2], scale_log2, -m_safe));
-        const float p3 = exp2f(fmaf(s[i + 3], scale_log2, -m_safe));
+      for (int i = 0; i < 64; i += 4) {
+        const float p0 = ex2(fmaf(s[i], scale_log2, -m_safe));
+        const float p1 = ex2(fmaf(s[i + 1], scale_log2, -m_safe));
+        const float p2 = ex2(fmaf(s[i + 2], scale_log2, -m_safe));
+        const float p3 = ex2(fmaf(s[i + 3], scale_log2, -m_safe));
         sum0 += p0; sum1 += p1; sum2 += p2; sum3 += p3;
         __nv_bfloat162 a = __floats2bfloat162_rn(p0, p1);
         __nv_bfloat162 bq = __floats2bfloat162_rn(p2, p3);
@@ -300,42 +330,48 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         tc::tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < 2; ++cc) {
             uint32_t v[32];
-            tc::tmem_ld32(tl + kColO + cc * 32, v);
+            const uint32_t col = kColO + half * 64 + cc * 32;
+            tc::tmem_ld32(tl + col, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tc::tmem_st32(tl + kColO + cc * 32, v);
+            tc::tmem_st32(tl + col, v);
           }
         }
       }
-      // P row -> shared memory, 128-byte swizzle: 16-byte chunk cc of row r at cc ^ (r & 7)
-      uint8_t* prow = sm + kSmemP + r * 128;
+      // this half of the P row -> shared memory, 128-byte swizzle: 16-byte chunk cc of
+      // row r at cc ^ (r & 7)
+      uint8_t* prow = sm + kSmemP + half * kHalf + r * 128;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const int w0 = half * 32 + cc * 4;
-          uint4 v4 = make_uint4(pk[w0], pk[w0 + 1], pk[w0 + 2], pk[w0 + 3]);
-          *reinterpret_cast<uint4*>(prow + half * kHalf + ((cc ^ (r & 7)) * 16)) = v4;
-        }
+      for (int cc = 0; cc < 8; ++cc) {
+        uint4 v4 = make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) * 16)) = v4;
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c.p_full);
     }
-    // epilogue
-    uint16_t* orow = out + ((size_t)bh * N + (size_t)t * BQ + r) * HD;
+    // epilogue: each half normalises and stores its 64 output columns
+    uint16_t* orow = out + ((size_t)bh * N + (size_t)t * BQ + r) * HD + half * 64;
     bool have = ok && ntiles > 0;
     if (have) have = warp_all(tc::mbar_wait(&c.o_ready, (ntiles - 1) & 1, abort_flag, dev_status));
+    if (ntiles > 0) {
+      // both halves form the same row sum, lpart[0] + lpart[1]
+      c.lpart[half][r] = l;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&c.lbar[quarter]);
+      if (have) have = warp_all(tc::mbar_wait(&c.lbar[quarter], 0, abort_flag, dev_status));
+    }
     if (have) {
       tc::tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float lt = c.lpart[0][r] + c.lpart[1][r];
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32];
-        tc::tmem_ld32(tl + kColO + cc * 32, v);
+        tc::tmem_ld32(tl + kColO + half * 64 + cc * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
           uint32_t w[4];
@@ -348,12 +384,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
           *reinterpret_cast<uint4*>(orow + cc * 32 + i) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      if (lse) lse[bh * N + (size_t)t * BQ + r] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (lse && half == 0)
+        lse[bh * N + (size_t)t * BQ + r] = lt > 0.f ? (m_used + log2f(lt)) * 0.69314718055994531f : -INFINITY;
     } else if (ntiles == 0) {
 #pragma unroll
-      for (int i = 0; i < HD; i += 8)
+      for (int i = 0; i < 64; i += 8)
         *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
-      if (lse) lse[bh * N + (size_t)t * BQ + r] = -INFINITY;
+      if (lse && half == 0) lse[bh * N + (size_t)t * BQ + r] = -INFINITY;
     }
   }
 

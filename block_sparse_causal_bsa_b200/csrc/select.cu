@@ -1,17 +1,18 @@
 // Per-tile top-k selection, the uncertainty gate and kv_idx
 // ([UGS] steps 2-5; [Stem] 2.A for the position-dependent budget).
 //
-// select_rank: one CTA per (b, h, tile). The candidate blocks 0..f_lo-1 are
-//   ranked by (score desc, index asc) with a bitonic sort of 64-bit keys in
-//   shared memory; the first `need` indices go to the ranked list, and the
-//   cut margin sigma = (s_(m-1) - s_(m)) / (s_(0) - s_(m)) is evaluated in
-//   fp32 with correctly rounded operations ([UGS] step 3).
+// select_rank: one warp per (b, h, tile). The candidate blocks 0..f_lo-1 are
+//   ranked by (score desc, index asc): exact radix selection on order-preserving
+//   32-bit keys finds the m-th and M-th largest, and one pass in block order
+//   writes the top-M blocks ascending, marking the top-m ones. The cut margin
+//   sigma = (s_(m-1) - s_(m)) / (s_(0) - s_(m)) is evaluated in fp32 with
+//   correctly rounded operations on the scores read back by index ([UGS] step 3).
 // gate: one CTA. sigma_bar[b,t] = fp32 sum of sigma over heads in head order,
 //   divided by Hq; theta = linear-interpolation empirical quantile of
 //   sigma_bar over the cut tiles of the call; trigger = cut && sigma_bar <
 //   theta ([UGS] step 4).
-// finalize: one CTA per (b, h, tile): forced blocks plus the first m_t (or
-//   M_t when triggered) ranked candidates, ascending, -1 padded to W
+// finalize: one warp per (b, h, tile): the first m_t (or M_t when triggered)
+//   ranked candidates, ascending, then the forced blocks, -1 padded to W
 //   ([UGS] step 5).
 #include <math.h>
 
@@ -45,70 +46,210 @@ __device__ void bitonic_sort(K* a, unsigned n, bool descending) {
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(512) select_rank_kernel(
-    const float* __restrict__ scores, int n_qt, int n_kb, int tile_q, int block_k, int k_first,
-    int k_last, int rho, int R, int32_t* __restrict__ ranked, float* __restrict__ sigma,
+// ---------------------------------------------------------------------------
+// Ranking: one warp per (b, h, tile) row, radix select on order-preserving
+// 32-bit keys in the warp's shared-memory slice.
+
+constexpr uint32_t kInTopM = 0x80000000u;   // flag on a ranked entry: inside the base top-m set
+
+struct RadixSel {
+  uint32_t v;      // key of the element at the requested rank
+  int take_eq;     // how many keys equal to v (lowest indices first) are inside the top r+1
+};
+
+// Key of the (r+1)-th largest among keys[0..n), n >= r+1. Digits of 8 bits, starting
+// below the bits every key of the row shares (so the first histogram spreads out).
+__device__ RadixSel warp_radix_select(const uint32_t* keys, int n, int r, uint32_t kmin, uint32_t kmax,
+                                      uint32_t* hist, int lane) {
+  int want = r + 1;
+  if (kmin == kmax) return {kmax, want};
+  const int hb = 31 - __clz(kmin ^ kmax);
+  uint32_t mask = hb == 31 ? 0u : ~((2u << hb) - 1u);
+  uint32_t prefix = kmax & mask;
+  int lo = hb + 1;
+  while (lo > 0) {
+    const int width = lo < 8 ? lo : 8;
+    const int shift = lo - width;
+    const uint32_t dmask = (1u << width) - 1u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) hist[lane * 8 + k] = 0u;
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+      const uint32_t u = keys[i];
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
+    }
+    __syncwarp();
+    uint32_t h8[8], s = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) { h8[k] = hist[lane * 8 + k]; s += h8[k]; }
+    uint32_t incl = s;                        // sum over lanes >= this lane
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+      if (lane + off < 32) incl += y;
+    }
+    uint32_t c = incl - s;                    // keys whose digit lies in higher lanes' bins
+    int found = -1;
+    uint32_t c_at = 0;
+#pragma unroll
+    for (int k = 7; k >= 0; --k) {
+      if (found < 0 && c < (uint32_t)want && (uint32_t)want <= c + h8[k]) { found = lane * 8 + k; c_at = c; }
+      c += h8[k];
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, found >= 0);
+    const int src = __ffs(bal) - 1;
+    const int dgt = __shfl_sync(0xffffffffu, found, src);
+    const uint32_t cd = __shfl_sync(0xffffffffu, c_at, src);
+    prefix |= (uint32_t)dgt << shift;
+    mask |= dmask << shift;
+    want -= (int)cd;
+    lo = shift;
+    __syncwarp();
+  }
+  return {prefix, want};
+}
+
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = max(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ uint32_t warp_min_u32(uint32_t x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = min(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ int warp_min_i32(int x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = min(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// Writes, per row, the top-M candidates (M = expanded slots) in ascending block
+// order with kInTopM set on the top-m ones (m = base slots; top-m is a prefix of
+// the same ranking, so it is a subset), and sigma from ranks 0, m-1, m.
+__global__ void __launch_bounds__(256) select_rank_kernel(
+    const float* __restrict__ scores, int rows_bh, int n_qt, int n_kb, int tile_q, int block_k,
+    int k_first, int k_last, int rho, int R, int32_t* __restrict__ ranked, float* __restrict__ sigma,
     int32_t* dev_status) {
-  extern __shared__ unsigned long long keys[];
+  extern __shared__ uint32_t wsm[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int wpc = blockDim.x / 32;
+  const int bh = blockIdx.y * wpc + warp;
+  if (bh >= rows_bh) return;
   const int t = blockIdx.x;
-  const size_t row = (size_t)blockIdx.y * n_qt + t;
+  uint32_t* keys = wsm + (size_t)warp * (n_kb + 256);
+  uint32_t* hist = keys + n_kb;
+  const size_t row = (size_t)bh * n_qt + t;
   const TileSlots sl = tile_slots(t, n_qt, tile_q, block_k, k_first, k_last, rho);
   const int n = sl.f_lo;
   const float* s = scores + row * n_kb;
   if (n == 0) {
-    if (threadIdx.x == 0) sigma[row] = 1.0f;
+    if (lane == 0) sigma[row] = 1.0f;
     return;
   }
-  int need = sl.M > sl.m ? sl.M : sl.m;
-  if (sl.cut && need < sl.m + 1) need = sl.m + 1;
-  if (need > n) need = n;
-  const unsigned P = next_pow2((unsigned)n);
-  __shared__ int bad;
-  if (threadIdx.x == 0) bad = 0;
-  __syncthreads();
-  for (unsigned i = threadIdx.x; i < P; i += blockDim.x) {
-    unsigned long long key = 0ull;            // padding sorts last
-    if (i < (unsigned)n) {
-      float x = s[i];
-      if (!isfinite(x)) bad = 1;
-      key = ((unsigned long long)score_key(x) << 32) | (unsigned long long)(~i);
-    }
-    keys[i] = key;
+  uint32_t kmax = 0u, kmin = 0xffffffffu;
+  bool bad = false;
+  for (int i = lane; i < n; i += 32) {
+    const float x = s[i];
+    bad |= !isfinite(x);
+    const uint32_t u = score_key(x);
+    keys[i] = u;
+    kmax = max(kmax, u);
+    kmin = min(kmin, u);
   }
-  bitonic_sort(keys, P, true);
+  kmax = warp_max_u32(kmax);
+  kmin = warp_min_u32(kmin);
+  bad = __any_sync(0xffffffffu, bad);
+  __syncwarp();
+  const int m = sl.m, M = sl.M;
+  RadixSel selm{0u, 0}, selM{0u, 0};
+  if (m > 0 && m < n) selm = warp_radix_select(keys, n, m - 1, kmin, kmax, hist, lane);
+  if (M > m && M < n) selM = warp_radix_select(keys, n, M - 1, kmin, kmax, hist, lane);
+  else if (M == m) selM = selm;
+  const bool all_m = m >= n, all_M = M >= n;
+
+  // one pass in block order: compaction of the top-M list, sigma bookkeeping
   int32_t* out = ranked + row * R;
-  for (int r = threadIdx.x; r < need; r += blockDim.x) out[r] = (int32_t)(~(uint32_t)keys[r]);
-  if (threadIdx.x == 0) {
-    if (bad) set_status(dev_status, BSA_DEV_BAD_SCORE);
-    float sg = 1.0f;
+  int base_M = 0, eq_m = 0, eq_M = 0;
+  int idx0 = 0x7fffffff, idx_m1 = 0x7fffffff, idx_eqnext = 0x7fffffff, idx_below = 0x7fffffff;
+  uint32_t below = 0u;
+  bool have_below = false;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int b0 = 0; b0 < n; b0 += 32) {
+    const int i = b0 + lane;
+    const bool live = i < n;
+    const uint32_t u = live ? keys[i] : 0u;
+    const bool e_m = live && !all_m && m > 0 && u == selm.v;
+    const unsigned bal_m = __ballot_sync(0xffffffffu, e_m);
+    const int r_m = eq_m + __popc(bal_m & lt);
+    const bool in_m = live && (all_m || (m > 0 && (u > selm.v || (e_m && r_m < selm.take_eq))));
+    const bool e_M = live && !all_M && u == selM.v;
+    const unsigned bal_M = __ballot_sync(0xffffffffu, e_M);
+    const int r_M = eq_M + __popc(bal_M & lt);
+    const bool in_M = live && M > 0 && (all_M || u > selM.v || (e_M && r_M < selM.take_eq));
+    const unsigned bal_in = __ballot_sync(0xffffffffu, in_M);
+    if (in_M) out[base_M + __popc(bal_in & lt)] = i | (in_m ? (int)kInTopM : 0);
+    base_M += __popc(bal_in);
+    if (live && u == kmax) idx0 = min(idx0, i);
+    if (sl.cut) {
+      if (e_m && r_m == selm.take_eq - 1) idx_m1 = i;
+      if (e_m && r_m == selm.take_eq) idx_eqnext = i;
+      if (live && u < selm.v && (!have_below || u > below || (u == below && i < idx_below))) {
+        below = u;
+        idx_below = i;
+        have_below = true;
+      }
+    }
+    eq_m += __popc(bal_m);
+    eq_M += __popc(bal_M);
+  }
+  idx0 = warp_min_i32(idx0);
+  float sg = 1.0f;
+  if (sl.cut) {
+    idx_m1 = warp_min_i32(idx_m1);
+    idx_eqnext = warp_min_i32(idx_eqnext);
+    // rank m: the next equal key if the top-m set left one out, else the best key below
+    int idx_m = idx_eqnext;
+    if (idx_m == 0x7fffffff) {
+      const uint32_t bmax = warp_max_u32(have_below ? below : 0u);
+      const bool mine = have_below && below == bmax;
+      idx_m = warp_min_i32(mine ? idx_below : 0x7fffffff);
+    }
+    const float s0 = s[idx0], a = s[idx_m1], b = s[idx_m];
+    const float num = __fsub_rn(a, b);
+    const float den = __fsub_rn(s0, b);
+    sg = (den == 0.0f) ? 0.0f : __fdiv_rn(num, den);
+  }
+  if (lane == 0) {
     if (bad) {
+      set_status(dev_status, BSA_DEV_BAD_SCORE);
       sg = __int_as_float(0x7fc00000);
-    } else if (sl.cut) {
-      // values read back from the score row, so signed zeros match the input exactly
-      float s0 = s[~(uint32_t)keys[0]];
-      float a = s[~(uint32_t)keys[sl.m - 1]];
-      float b = s[~(uint32_t)keys[sl.m]];
-      float num = __fsub_rn(a, b);
-      float den = __fsub_rn(s0, b);
-      sg = (den == 0.0f) ? 0.0f : __fdiv_rn(num, den);
     }
     sigma[row] = sg;
   }
+}
+
+static int rank_warps_per_cta(int n_kb) {
+  const size_t per_warp = ((size_t)n_kb + 256) * 4;
+  int w = (int)((96u * 1024u) / per_warp);
+  return w < 1 ? 1 : (w > 8 ? 8 : w);
 }
 
 cudaError_t launch_select_rank(const bsa_shape& s, const bsa_select_params& p, const float* scores,
                                int R, int32_t* ranked, float* sigma, int32_t* dev_status,
                                cudaStream_t st) {
   const int n_qt = s.N / s.tile_q, n_kb = s.N / s.block_k;
-  unsigned P = 1;
-  while (P < (unsigned)n_kb) P <<= 1;
-  size_t smem = (size_t)P * 8;
+  const int wpc = rank_warps_per_cta(n_kb);
+  const size_t smem = (size_t)wpc * (n_kb + 256) * 4;
   cudaError_t e = cudaFuncSetAttribute(select_rank_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(n_qt, s.B * s.Hq);
-  select_rank_kernel<<<grid, 512, smem, st>>>(scores, n_qt, n_kb, s.tile_q, s.block_k, p.k_first,
-                                              p.k_last, p.rho, R, ranked, sigma, dev_status);
+  const int rows_bh = s.B * s.Hq;
+  dim3 grid(n_qt, (rows_bh + wpc - 1) / wpc);
+  select_rank_kernel<<<grid, wpc * 32, smem, st>>>(scores, rows_bh, n_qt, n_kb, s.tile_q, s.block_k,
+                                                   p.k_first, p.k_last, p.rho, R, ranked, sigma,
+                                                   dev_status);
   return cudaGetLastError();
 }
 
@@ -180,45 +321,46 @@ cudaError_t launch_gate(const bsa_shape& s, const bsa_select_params& p, const fl
 
 // ---------------------------------------------------------------------------
 
+// One warp per (b, h, tile) row: the triggered tiles take the whole top-M list,
+// the others only its kInTopM entries; both are already in ascending block
+// order and precede the forced blocks, which follow; -1 pads to W.
 __global__ void __launch_bounds__(256) finalize_kernel(
-    const int32_t* __restrict__ ranked, int R, const uint8_t* __restrict__ trigger, int Hq,
-    int n_qt, int tile_q, int block_k, int k_first, int k_last, int rho, int W,
+    const int32_t* __restrict__ ranked, int R, const uint8_t* __restrict__ trigger, int rows_bh,
+    int Hq, int n_qt, int tile_q, int block_k, int k_first, int k_last, int rho, int W,
     int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt) {
-  extern __shared__ int32_t buf[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bh = blockIdx.y * (blockDim.x / 32) + warp;
+  if (bh >= rows_bh) return;
   const int t = blockIdx.x;
-  const int bh = blockIdx.y;
   const int b = bh / Hq;
   const size_t row = (size_t)bh * n_qt + t;
   const TileSlots sl = tile_slots(t, n_qt, tile_q, block_k, k_first, k_last, rho);
-  const int take = trigger[(size_t)b * n_qt + t] ? sl.M : sl.m;
-  const unsigned P = next_pow2((unsigned)(take > 0 ? take : 1));
-  for (unsigned i = threadIdx.x; i < P; i += blockDim.x)
-    buf[i] = (int)i < take ? ranked[row * R + i] : 0x7fffffff;
-  bitonic_sort(buf, P, false);
+  const bool all = trigger[(size_t)b * n_qt + t] != 0;
+  const int take = all ? sl.M : sl.m;
+  const int32_t* in = ranked + row * R;
   int32_t* out = kv_idx + row * W;
-  for (int i = threadIdx.x; i < W; i += blockDim.x) {
-    int32_t x;
-    if (i < take) x = buf[i];
-    else if (i < take + sl.nF) x = sl.f_lo + (i - take);
-    else x = -1;
-    out[i] = x;
+  const unsigned lt = (1u << lane) - 1u;
+  int pos = 0;
+  for (int b0 = 0; b0 < sl.M; b0 += 32) {
+    const int i = b0 + lane;
+    const int32_t e = i < sl.M ? in[i] : 0;
+    const bool keep = i < sl.M && (all || (e & (int32_t)kInTopM));
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[pos + __popc(bal & lt)] = e & 0x7fffffff;
+    pos += __popc(bal);
   }
-  if (threadIdx.x == 0) kv_cnt[row] = take + sl.nF;
+  for (int i = take + lane; i < W; i += 32) out[i] = (i < take + sl.nF) ? sl.f_lo + (i - take) : -1;
+  if (lane == 0) kv_cnt[row] = take + sl.nF;
 }
 
 cudaError_t launch_finalize(const bsa_shape& s, const bsa_select_params& p, const int32_t* ranked,
                             int R, const uint8_t* trigger, int W, int32_t* kv_idx, int32_t* kv_cnt,
                             cudaStream_t st) {
   const int n_qt = s.N / s.tile_q;
-  unsigned P = 1;
-  while (P < (unsigned)W) P <<= 1;
-  size_t smem = (size_t)P * 4;
-  cudaError_t e = cudaFuncSetAttribute(finalize_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(n_qt, s.B * s.Hq);
-  finalize_kernel<<<grid, 256, smem, st>>>(ranked, R, trigger, s.Hq, n_qt, s.tile_q, s.block_k,
-                                           p.k_first, p.k_last, p.rho, W, kv_idx, kv_cnt);
+  const int rows_bh = s.B * s.Hq;
+  dim3 grid(n_qt, (rows_bh + 7) / 8);
+  finalize_kernel<<<grid, 256, 0, st>>>(ranked, R, trigger, rows_bh, s.Hq, n_qt, s.tile_q, s.block_k,
+                                        p.k_first, p.k_last, p.rho, W, kv_idx, kv_cnt);
   return cudaGetLastError();
 }
 
