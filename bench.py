@@ -242,6 +242,27 @@ def cpu_baseline(spec, seed, target_s=15.0):
 # ---------------------------------------------------------------------------
 # GPU arm
 
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own independent problem (weak scaling)."""
+    return 1003 + 1000 * rank
+
+
+def reduce_over_ranks(step_ms, attend_ms, e2e_ms, flops, world, device):
+    """Max of the per-rank times and sum of the per-rank work (the slowest rank sets
+    the job's time; value = all ranks' work / that time). No data moves between
+    ranks on the compute path; this is the only collective besides the barriers."""
+    import torch
+    t = torch.tensor([step_ms, attend_ms, e2e_ms, flops], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        mx = t.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        tot = t.clone()
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+        return float(mx[0]), float(mx[1]), float(mx[2]), float(tot[3])
+    return step_ms, attend_ms, e2e_ms, flops
+
+
 def _dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -263,7 +284,7 @@ def main_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
     spec = S.WORKLOADS[WORKLOAD]
-    seed = 1003 + 1000 * rank
+    seed = rank_seed(rank)
     qh, kh, vh = _gen_prefill(spec, seed)
     q, k, v = _bf16(torch, qh, dev), _bf16(torch, kh, dev), _bf16(torch, vh, dev)
     stream = torch.cuda.current_stream(dev)
@@ -391,16 +412,8 @@ def main_gpu(args):
     dec["peak_note"] = f"{peak_kind} HBM {peaks['hbm_gbs']} GB/s"
 
     # max over ranks
-    t = torch.tensor([step_ms, attend_ms, e2e_ms, flops], dtype=torch.float64, device=dev)
-    if world > 1:
-        mx = t.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        tot = t.clone()
-        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
-        step_ms, attend_ms, e2e_ms = float(mx[0]), float(mx[1]), float(mx[2])
-        total_flops = float(tot[3])
-    else:
-        total_flops = flops
+    step_ms, attend_ms, e2e_ms, total_flops = reduce_over_ranks(step_ms, attend_ms, e2e_ms, flops,
+                                                                world, dev)
     if rank == 0:
         sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         achieved = flops / (attend_ms * 1e-3) / 1e12

@@ -25,8 +25,9 @@ Workloads (sizes and structure of the pages' settings):
 * ``gated_prefill_128k``: B=1, 32/8 heads, N=131072, d=128, block 64, tile
   128, base k=64, rho=2, quantile 0.25. K rows are a per-block mean plus
   unit noise; adjacent block pairs (2m, 2m+1) become twins with probability
-  ``p_twin`` (exact copies, or copies with one element moved by one bf16
-  ulp), which plants near-tied block scores at the top-k cut.
+  ``p_twin`` = 0.36 (exact copies, or copies with one element moved by one
+  bf16 ulp), which plants near-tied block scores at the top-k cut: about a
+  fifth of the (head, cut tile) pairs then have s_(k-1) - s_(k) < 1e-3.
 * ``tpd_oam_prefill_64k``: B=2, 32/8 heads, N=65536, d=128, block 64, tile
   128, k decaying linearly from 128 to 32, output-aware score; V rows are
   exp(N(0,1)) * N(0, I) (log-normal row norms, sigma=1).
@@ -121,7 +122,7 @@ WORKLOADS = {
     "gated_prefill_128k": PrefillSpec(
         "gated_prefill_128k", B=1, Hq=32, Hkv=8, N=131072, d=128, block_k=64,
         tile_q=128, k_first=64, k_last=64, rho=2, gate_quantile=0.25,
-        score_kind="mean", dtype="bf16", structure="twins", p_twin=0.25,
+        score_kind="mean", dtype="bf16", structure="twins", p_twin=0.36,
         block_mean_std=1.0),
     "tpd_oam_prefill_64k": PrefillSpec(
         "tpd_oam_prefill_64k", B=2, Hq=32, Hkv=8, N=65536, d=128, block_k=64,

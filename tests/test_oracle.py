@@ -490,3 +490,25 @@ def test_attend_empty_rows():
     # tile 1 listing only block 2, which is after every row of the tile
     o, l = O.attend_tile(Q[64:128], K, V, np.array([2]), 64, bk, 0.3)
     assert (o == 0).all() and np.isneginf(l).all()
+
+
+def test_gated_workload_near_tie_fraction():
+    """The 128k gated workload is drawn so that about a fifth of the (head, cut
+    tile) pairs have a gap below 1e-3 between the last kept and the first dropped
+    candidate score (oracle scores; every 4th tile of all 32 heads)."""
+    spec = S.WORKLOADS["gated_prefill_128k"]
+    G = spec.Hq // spec.Hkv
+    near = tot = 0
+    for g in range(spec.Hkv):
+        kb = O.pool_keys(S.prefill_head(spec, 1003, "k", 0, g), spec.block_k)
+        for h in range(g * G, (g + 1) * G):
+            q = S.prefill_head(spec, 1003, "q", 0, h)
+            for t in range(1 + (h % 4), spec.n_qt, 4):
+                nF, nc, m, M = O.tile_slots(t, spec.n_qt, spec.tile_q, spec.block_k, 64, 64, 2)
+                if not nc > m >= 1:
+                    continue
+                s = O.score_tile(q[t * 128:(t + 1) * 128], kb, O.tile_blocks(t, 128, 64)[1])
+                o = O.rank_candidates(s, nc)
+                near += float(s[o[m - 1]]) - float(s[o[m]]) < 1e-3
+                tot += 1
+    assert 0.15 <= near / tot <= 0.25, near / tot
