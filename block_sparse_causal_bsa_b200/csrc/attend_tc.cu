@@ -10,24 +10,27 @@
 //   warp 0 (one thread)  TMA producer: the Q tile once, then K and V tiles of
 //                        128 keys = two listed blocks gathered into adjacent
 //                        shared-memory rows, two stages deep.
-//   warp 1 (one thread)  MMA issuer: S_j = Q K_j^T into one of two TMEM
-//                        buffers, then O += P_j V_j into the TMEM accumulator.
-//                        S_{j+1} is issued before PV_j so the tensor core
-//                        works while the softmax warps handle tile j.
+//   warp 1 (one thread)  MMA issuer: S_j = Q K_j^T into one of two TMEM buffers
+//                        (S_{j+1} is issued before the value products of tile j),
+//                        then, per half tile (one listed block), O_h += P_h V_h
+//                        into that half's own TMEM accumulator as soon as the
+//                        half's P is written.
 //   warps 2-9            softmax: two warps per TMEM lane quarter; a thread owns
-//                        half of one query row (64 of the tile's 128 keys, i.e.
-//                        one listed block). The two halves of a row exchange
-//                        their tile max through shared memory (a 64-thread
-//                        named barrier per lane quarter), then each applies the
-//                        causal mask on the diagonal tile, exponentiates, keeps
-//                        its part of the row sum, writes its half of P_j (bf16)
-//                        into 128-byte-swizzled shared memory, and rescales its
-//                        half of the O row in TMEM only when the running max
-//                        grew by more than 2^8 (exact: the final division uses
-//                        the same max). Epilogue: O / l -> bf16, optional lse.
+//                        half of one query row (the 64 keys of one listed block)
+//                        and runs an independent online softmax over the blocks
+//                        it sees: running max and sum of its half only, its own
+//                        O_h accumulator, rescaled in TMEM only when its running
+//                        max grew by more than 2^8 (exact: l and O keep the same
+//                        stale max). No per-tile exchange between the halves.
+//                        Epilogue: the two halves meet once, through shared
+//                        memory: m = max(m0, m1), l = l0 2^(m0-m) + l1 2^(m1-m),
+//                        O = (O_0 2^(m0-m) + O_1 2^(m1-m)) / l  -- the exact merge
+//                        of two softmax partial sums; each half writes 64 of the
+//                        128 output columns (and lse).
 // Operand layouts (all 128-byte swizzled, as TMA writes them):
 //   Q, K: K-major [rows x 64 elements] halves; P: K-major (keys are K);
 //   V: MN-major (rows = keys, 64 contiguous head dims per 128-byte row).
+// TMEM: S buffers at columns 0 and 128, O_0 at 256, O_1 at 384.
 // The CTA-to-work mapping walks (batch, KV head) outermost and the query heads
 // of a group innermost, so CTAs running together gather from one KV head and
 // reuse its blocks through L2.
@@ -55,20 +58,20 @@ constexpr uint32_t kTile = 2 * kHalf;        // 128 rows x 128 dims bf16
 constexpr uint32_t kBoxK = 8192;             // one 64-key block half
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;                // S buffers at columns 0 and 128
-constexpr uint32_t kColO = 256;              // O accumulator
+constexpr uint32_t kColO = 256;              // O_0 at 256, O_1 at 384
 
 struct __align__(8) Ctrl {
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, o_ready, done;
+  uint64_t p_full[2], o_ready[2];   // per half tile
+  uint64_t done;
+  uint64_t lbar[4];                 // per lane quarter: both halves' (m, l) written (once)
   uint32_t tmem;
   int abort_flag;
   int n_list;
-  uint64_t xbar[4];          // per lane quarter: both half-row maxima written (one phase per tile)
-  uint64_t lbar[4];          // per lane quarter: both row-sum parts written (once)
-  float xmax[2][2][128];     // [tile parity][half][row] max of the half-row
-  float lpart[2][128];       // [half][row] row-sum part
+  float mpart[2][128];              // [half][row] final running max of the half
+  float lpart[2][128];              // [half][row] final row-sum part of the half
   int list[kMaxList];
 };
 
@@ -127,13 +130,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&c.s_full[i], 1);
       tc::mbar_init(&c.s_free[i], kSoftmaxWarps);
+      tc::mbar_init(&c.p_full[i], kSoftmaxWarps / 2);
+      tc::mbar_init(&c.o_ready[i], 1);
     }
-    tc::mbar_init(&c.p_full, kSoftmaxWarps);
-    for (int q = 0; q < 4; ++q) {
-      tc::mbar_init(&c.xbar[q], 2);
-      tc::mbar_init(&c.lbar[q], 2);
-    }
-    tc::mbar_init(&c.o_ready, 1);
+    for (int q = 0; q < 4; ++q) tc::mbar_init(&c.lbar[q], 2);
     tc::mbar_init(&c.done, 1);
     c.abort_flag = 0;
     tc::fence_mbar_init();
@@ -233,18 +233,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         tc::tc_fence_after();
         issue_s(jn);
       }
-      ok = tc::mbar_wait(&c.p_full, j & 1, abort_flag, dev_status) &&
-           tc::mbar_wait(&c.v_full[j % NS], (j / NS) & 1, abort_flag, dev_status);
+      ok = tc::mbar_wait(&c.v_full[j % NS], (j / NS) & 1, abort_flag, dev_status);
       if (!ok) break;
-      tc::tc_fence_after();
       const uint32_t vb = sV + (j % NS) * kTile;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t aoff = (kk >> 2) * kHalf + (kk & 3) * 32;
-        tc::umma_bf16(tmem + kColO, tc::sdesc_sw128(sP + aoff, 16, 1024),
-                      tc::sdesc_sw128(vb + kk * 2048, kHalf, 1024), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+      for (int half = 0; half < 2; ++half) {
+        ok = tc::mbar_wait(&c.p_full[half], j & 1, abort_flag, dev_status);
+        if (!ok) break;
+        tc::tc_fence_after();
+        // O_half += P_half (128 rows x 64 keys) . V rows of this half's block
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          tc::umma_bf16(tmem + kColO + half * 128, tc::sdesc_sw128(sP + half * kHalf + kk * 32, 16, 1024),
+                        tc::sdesc_sw128(vb + (half * 4 + kk) * 2048, kHalf, 1024), idPV,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::umma_commit(&c.o_ready[half]);
       }
-      tc::umma_commit(&c.o_ready);
+      if (!ok) break;
       tc::umma_commit(&c.v_empty[j % NS]);
     }
   } else if (warp >= 2) {
@@ -253,9 +259,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const int half = (warp - 2) >> 2;                   // 0: keys 0-63 of the tile, 1: keys 64-127
     const int r = quarter * 32 + lane;                  // row in the tile == TMEM lane
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t colO = kColO + half * 128;
     const int row_abs = t * BQ + r;
-    float m_used = -INFINITY;                           // running max, scaled log2 units
-    float l = 0.f;                                      // this half's part of the row sum
+    float m_used = -INFINITY;                           // running max of this half, scaled log2 units
+    float l = 0.f;                                      // running sum of this half
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       ok = warp_all(tc::mbar_wait(&c.s_full[j % 2], (j / 2) & 1, abort_flag, dev_status));
@@ -291,16 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 #pragma unroll
         for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
       }
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // share the half-row max with the partner warp (buffer alternates by tile parity;
-      // a buffer is rewritten two tiles later, after the partner passed the next exchange)
-      c.xmax[j & 1][half][r] = mx;
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&c.xbar[quarter]);
-      ok = warp_all(tc::mbar_wait(&c.xbar[quarter], j & 1, abort_flag, dev_status));
-      if (!ok) break;
-      mx = fmaxf(mx, c.xmax[j & 1][half ^ 1][r]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * scale_log2;
       float alpha = 1.f;
       if (m_tile > m_used + 8.0f) {                     // also taken when m_used is -inf
@@ -325,18 +324,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
       l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
 
       if (j > 0) {
-        ok = warp_all(tc::mbar_wait(&c.o_ready, (j - 1) & 1, abort_flag, dev_status));
+        // the previous value product of this half has read P_half and updated O_half
+        ok = warp_all(tc::mbar_wait(&c.o_ready[half], (j - 1) & 1, abort_flag, dev_status));
         if (!ok) break;
         tc::tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
+          for (int cc = 0; cc < 4; ++cc) {
             uint32_t v[32];
-            const uint32_t col = kColO + half * 64 + cc * 32;
-            tc::tmem_ld32(tl + col, v);
+            tc::tmem_ld32(tl + colO + cc * 32, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tc::tmem_st32(tl + col, v);
+            tc::tmem_st32(tl + colO + cc * 32, v);
           }
         }
       }
@@ -351,41 +350,51 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&c.p_full);
+      if (lane == 0) tc::mbar_arrive(&c.p_full[half]);
     }
-    // epilogue: each half normalises and stores its 64 output columns
+    // epilogue: merge the two halves' partial softmax sums, store 64 columns each
     uint16_t* orow = out + ((size_t)bh * N + (size_t)t * BQ + r) * HD + half * 64;
     bool have = ok && ntiles > 0;
-    if (have) have = warp_all(tc::mbar_wait(&c.o_ready, (ntiles - 1) & 1, abort_flag, dev_status));
+    if (have) have = warp_all(tc::mbar_wait(&c.o_ready[half], (ntiles - 1) & 1, abort_flag, dev_status));
     if (ntiles > 0) {
-      // both halves form the same row sum, lpart[0] + lpart[1]
+      c.mpart[half][r] = m_used;
       c.lpart[half][r] = l;
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c.lbar[quarter]);
+      // each half arrives only after its own last value product completed, so past
+      // this barrier both O accumulators are final
       if (have) have = warp_all(tc::mbar_wait(&c.lbar[quarter], 0, abort_flag, dev_status));
     }
     if (have) {
       tc::tc_fence_after();
-      const float lt = c.lpart[0][r] + c.lpart[1][r];
+      const float m0 = c.mpart[0][r], m1 = c.mpart[1][r];
+      const float mm = fmaxf(m0, m1);
+      const float f0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - mm);
+      const float f1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - mm);
+      const float lt = c.lpart[0][r] * f0 + c.lpart[1][r] * f1;
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float w0 = f0 * inv, w1 = f1 * inv;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v[32];
-        tc::tmem_ld32(tl + kColO + half * 64 + cc * 32, v);
+        uint32_t v0[32], v1[32];
+        tc::tmem_ld32(tl + kColO + half * 64 + cc * 32, v0);          // O_0, this half's columns
+        tc::tmem_ld32(tl + kColO + 128 + half * 64 + cc * 32, v1);    // O_1, same columns
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 p = __floats2bfloat162_rn(__uint_as_float(v[i + 2 * e]) * inv,
-                                                     __uint_as_float(v[i + 2 * e + 1]) * inv);
+            const int k0 = i + 2 * e;
+            __nv_bfloat162 p = __floats2bfloat162_rn(
+                __uint_as_float(v0[k0]) * w0 + __uint_as_float(v1[k0]) * w1,
+                __uint_as_float(v0[k0 + 1]) * w0 + __uint_as_float(v1[k0 + 1]) * w1);
             w[e] = *reinterpret_cast<uint32_t*>(&p);
           }
           *reinterpret_cast<uint4*>(orow + cc * 32 + i) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       if (lse && half == 0)
-        lse[bh * N + (size_t)t * BQ + r] = lt > 0.f ? (m_used + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+        lse[bh * N + (size_t)t * BQ + r] = lt > 0.f ? (mm + log2f(lt)) * 0.69314718055994531f : -INFINITY;
     } else if (ntiles == 0) {
 #pragma unroll
       for (int i = 0; i < 64; i += 8)
@@ -400,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
   if (warp == 0 && lane == 0 && ntiles > 0) {
     // make sure no TMA copy of this CTA is still landing in shared memory: wait for
     // the last phase issued on every stage (earlier phases completed before it)
+    tc::mbar_wait_timed(&c.q_full, 0);
     for (int j = k_issued - NS < 0 ? 0 : k_issued - NS; j < k_issued; ++j)
       tc::mbar_wait_timed(&c.k_full[j % NS], (j / NS) & 1);
     for (int j = v_issued - NS < 0 ? 0 : v_issued - NS; j < v_issued; ++j)

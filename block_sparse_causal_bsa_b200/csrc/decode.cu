@@ -1,4 +1,6 @@
-// Decode attention with run-time termination ([ART] 2.1-2.4).
+// Decode attention with run-time termination ([ART] 2.1-2.4), CUDA-core kernel:
+// serves the shapes the tensor-core decode (decode_tc.cu) does not take
+// (d = 64, KV blocks of 64).
 //
 // One CTA per (batch, KV head). The CTA streams the KV cache in blocks of
 // block_kv keys, in order ([ART] 2.1: tile-wise streaming exposes the partial
@@ -23,14 +25,6 @@
 #include "kernels.h"
 
 namespace bsa {
-
-struct DecodeArgs {
-  int L, block_kv, Hq, Hkv;
-  float scale_log2;
-  float tau, phi;
-  int patience, enable, n_probe;
-  int dims[kMaxProbe];
-};
 
 namespace {
 constexpr int kStages = 3;
@@ -258,13 +252,15 @@ cudaError_t launch_decode(const bsa_decode_shape& s, const bsa_decode_params& p,
                           const void* kc, const void* vc, float scale, void* out,
                           int32_t* blocks_used, float* probe_trace, int32_t* dev_status,
                           cudaStream_t st) {
-  (void)dev_status;   // the decode kernel has no bounded waits or data-dependent indices
+  // the CUDA-core kernel below has no mbarrier waits and no data-dependent indices
   DecodeArgs a;
   a.L = s.L; a.block_kv = s.block_kv; a.Hq = s.Hq; a.Hkv = s.Hkv;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.tau = p.tau; a.phi = p.phi; a.patience = p.patience; a.enable = p.enable;
   a.n_probe = p.n_probe;
   for (int i = 0; i < kMaxProbe; ++i) a.dims[i] = i < p.n_probe ? p.probe_dims[i] : 0;
+  if (decode_tc_supported(s))
+    return launch_decode_tc(s, a, q, kc, vc, out, blocks_used, probe_trace, dev_status, st);
   const int G = s.Hq / s.Hkv;
 #define BSA_DEC(D)                                                                             \
   switch (G) {                                                                                 \

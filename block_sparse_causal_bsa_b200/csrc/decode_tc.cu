@@ -1,0 +1,408 @@
+// Decode attention with run-time termination on Blackwell tensor cores
+// ([ART] 2.1-2.4): the KV cache of one (batch, KV head) is streamed block by
+// block, in order; after each block the normalised partial output O^(t) is
+// probed, and from block 1 on the stability test decides whether to stop.
+//
+// One CTA per (batch, KV head), 224 threads:
+//   warp 0 (one thread)  TMA producer: K and V blocks of 128 keys, a ring of
+//                        three stages (64 KB each), until told to halt.
+//   warp 1 (one thread)  MMA issuer: S_t = K_t Q^T (M = 128 keys, N = 16: the
+//                        group's query heads padded with zero rows) into one of
+//                        two TMEM buffers; after the softmax warps publish P_t,
+//                        D_t = V_t^T P_t^T (M = 128 head dims, V_t read as an
+//                        MN-major operand straight from its TMA tile).
+//   warps 2-5            softmax and fold: a thread owns TMEM lane r, i.e. key r of
+//                        S_t and head dim r of D_t. Per head: the block max across
+//                        the four warps (shared memory + a bounded mbarrier
+//                        handshake), P_t to shared memory (bf16, 128-byte swizzle),
+//                        then O[h][r] = O[h][r] * alpha_h + D_t[r][h] in registers;
+//                        each warp keeps its own part of the row sums l.
+//   warp 6 (one thread)  decider: for block t it forms the probe
+//                        x^(t) = O^(t)[first head][probe dims] / l (fp32; l = the
+//                        four warp parts added in a fixed order) and runs the fp64
+//                        stability test (sums in index order, separate multiply and
+//                        add), then publishes stop / continue.
+// The work is software-pipelined: the MMA issuer computes S_{t+1} before PV_t,
+// and the softmax warps produce P_{t+1} (two P buffers) before they fold D_t, so
+// the softmax of one block overlaps the value product of the previous one. The
+// decider judges block t while the softmax warps go on; they look at that
+// verdict only before folding D_{t+1}, and on a stop return the unfolded O^(t). After a stop the producer
+// and MMA threads are released through a halt flag; the CTA then waits for its
+// own copies and MMAs and frees TMEM. All waits are bounded.
+// Shapes: bf16, d = 128, KV blocks of 128, Hq/Hkv <= 8.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace bsa {
+
+namespace {
+constexpr int HD = 128;
+constexpr int BKV = 128;
+constexpr int NPAD = 16;
+constexpr int GMAX = 8;
+constexpr int STAGES = 3;
+constexpr int kThreads = 224;
+constexpr uint32_t kHalf = 16384;         // 128 rows x 128 bytes
+constexpr uint32_t kTile = 2 * kHalf;     // one K or V block
+constexpr uint32_t kStage = 2 * kTile;    // K + V
+constexpr uint32_t kSmallHalf = 2048;     // 16 rows x 128 bytes
+constexpr uint32_t kTmemCols = 64;        // S[2] at 0/16, D[2] at 32/48
+
+struct __align__(8) Ctrl {
+  uint64_t kv_full[STAGES], kv_empty[STAGES];
+  uint64_t s_full[2], o_full[2];
+  uint64_t red_max, p_ready[2], probe_rdy, decided, done;
+  uint32_t tmem;
+  int abort_flag;     // error: softmax warps unwind
+  int halt;           // producer / MMA stop issuing (normal stop or error)
+  int stop_at;        // block after which the decider stopped, or -1
+  float rmax[2][4][GMAX];       // [block parity][warp][head]
+  float lpart[2][4];            // [block parity][warp] row-sum part of the first head
+  float xfull[2][HD];           // [block parity][head dim] unnormalised O of the first head
+  float lfin[4][GMAX];          // [warp][head] final row-sum parts
+  float xprev[kMaxProbe];
+};
+
+constexpr size_t kSmemStages = 0;
+constexpr size_t kSmemQ = kSmemStages + STAGES * kStage;
+constexpr size_t kSmemP = kSmemQ + 2 * kSmallHalf;            // two P buffers of 4 KB
+constexpr size_t kSmemCtrl = kSmemP + 4 * kSmallHalf;
+constexpr size_t kSmemBytes = kSmemCtrl + sizeof(Ctrl) + 1024;
+
+__device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// byte offset of element (row, col) in a 128-byte-swizzled K-major [rows x 128] operand
+// stored as two 64-column halves of half_bytes each
+__device__ __forceinline__ uint32_t sw128_off(int row, int col, uint32_t half_bytes) {
+  const int half = col >> 6, c = col & 63;
+  return half * half_bytes + row * 128 + ((((c >> 3) ^ (row & 7)) & 7) << 4) + (c & 7) * 2;
+}
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
+    const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+    const uint16_t* __restrict__ q, const DecodeArgs a, uint16_t* __restrict__ out,
+    int32_t* __restrict__ blocks_used, float* __restrict__ probe_trace, int32_t* dev_status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl& c = *reinterpret_cast<Ctrl*>(sm + kSmemCtrl);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bg = blockIdx.x;
+  const int b = bg / a.Hkv, g = bg % a.Hkv;
+  const int G = a.Hq / a.Hkv;
+  const int nb = a.L / BKV;
+  const int row0 = bg * a.L;
+  const uint32_t sStages = tc::smem_u32(sm + kSmemStages);
+  const uint32_t sQ = tc::smem_u32(sm + kSmemQ);
+  const uint32_t sP = tc::smem_u32(sm + kSmemP);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&c.kv_full[s], 1);
+      tc::mbar_init(&c.kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&c.s_full[i], 1);
+      tc::mbar_init(&c.o_full[i], 1);
+    }
+    tc::mbar_init(&c.red_max, 4);
+    tc::mbar_init(&c.p_ready[0], 4);
+    tc::mbar_init(&c.p_ready[1], 4);
+    tc::mbar_init(&c.probe_rdy, 4);
+    tc::mbar_init(&c.decided, 1);
+    tc::mbar_init(&c.done, 1);
+    c.abort_flag = 0;
+    c.halt = 0;
+    c.stop_at = -1;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&c.tmem, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (warp >= 2 && warp <= 5) {
+    // Q rows of the group (zero rows up to 16) and an all-zero P, both as K-major
+    // 128-byte-swizzled MMA operands
+    const int tid = threadIdx.x - 64;
+    uint32_t* qz = reinterpret_cast<uint32_t*>(sm + kSmemQ);
+    for (int i = tid; i < (int)(6 * kSmallHalf / 4); i += 128) qz[i] = 0u;   // Q and both P buffers
+    __syncwarp();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const uint16_t* qg = q + ((size_t)b * a.Hq + (size_t)g * G) * HD;
+    for (int e = tid; e < G * HD; e += 128) {
+      const int h = e / HD, col = e % HD;
+      *reinterpret_cast<uint16_t*>(sm + kSmemQ + sw128_off(h, col, kSmallHalf)) = qg[e];
+    }
+    tc::fence_proxy_async_smem();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = c.tmem;
+  volatile int* abort_flag = &c.abort_flag;
+  volatile int* halt = &c.halt;
+  int issued = 0;
+  bool mma_issued = false;
+  float o_fin[GMAX];        // softmax warps: unnormalised output of this thread's head dim
+  bool out_ok = false;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    tc::prefetch_tmap(&tmk);
+    tc::prefetch_tmap(&tmv);
+    for (int t = 0; t < nb; ++t) {
+      const int s = t % STAGES;
+      if (t >= STAGES && !tc::mbar_wait_halt(&c.kv_empty[s], ((t / STAGES) - 1) & 1, halt, dev_status)) break;
+      if (*halt) break;
+      uint8_t* st = sm + kSmemStages + s * kStage;
+      const int r = row0 + t * BKV;
+      tc::mbar_arrive_expect_tx(&c.kv_full[s], kStage);
+      tc::tma_load_2d(st, &tmk, 0, r, &c.kv_full[s]);
+      tc::tma_load_2d(st + kHalf, &tmk, 64, r, &c.kv_full[s]);
+      tc::tma_load_2d(st + kTile, &tmv, 0, r, &c.kv_full[s]);
+      tc::tma_load_2d(st + kTile + kHalf, &tmv, 64, r, &c.kv_full[s]);
+      issued = t + 1;
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    constexpr uint32_t idS = tc::idesc_bf16_f32(128, NPAD, false, false);
+    constexpr uint32_t idD = tc::idesc_bf16_f32(128, NPAD, true, false);
+    auto issue_s = [&](int t) -> bool {
+      const int s = t % STAGES;
+      if (!tc::mbar_wait_halt(&c.kv_full[s], (t / STAGES) & 1, halt, dev_status)) return false;
+      tc::tc_fence_after();
+      const uint32_t kb = sStages + s * kStage;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+        const uint32_t qoff = (kk >> 2) * kSmallHalf + (kk & 3) * 32;
+        tc::umma_bf16(tmem + (t & 1) * NPAD, tc::sdesc_sw128(kb + off, 16, 1024),
+                      tc::sdesc_sw128(sQ + qoff, 16, 1024), idS, kk > 0);
+      }
+      tc::umma_commit(&c.s_full[t & 1]);
+      mma_issued = true;
+      return true;
+    };
+    bool ok = issue_s(0);
+    for (int t = 0; ok && t < nb; ++t) {
+      // S_{t+1} first: its buffer held S_{t-1}, which the softmax warps read before P_{t-1}
+      if (t + 1 < nb && !issue_s(t + 1)) break;
+      if (!tc::mbar_wait_halt(&c.p_ready[t & 1], (t >> 1) & 1, halt, dev_status)) break;
+      tc::tc_fence_after();
+      const int s = t % STAGES;
+      const uint32_t vb = sStages + s * kStage + kTile;
+      const uint32_t pb = sP + (t & 1) * 2 * kSmallHalf;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t poff = (kk >> 2) * kSmallHalf + (kk & 3) * 32;
+        tc::umma_bf16(tmem + 32 + (t & 1) * NPAD, tc::sdesc_sw128(vb + kk * 2048, kHalf, 1024),
+                      tc::sdesc_sw128(pb + poff, 16, 1024), idD, kk > 0);
+      }
+      tc::umma_commit(&c.o_full[t & 1]);
+      tc::umma_commit(&c.kv_empty[s]);
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ---------------- softmax and fold ----------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;           // key of S_t, head dim of D_t
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    float m[GMAX], lw[GMAX], o[GMAX];
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) { m[h] = -INFINITY; lw[h] = 0.f; o[h] = 0.f; }
+    // softmax of block t: writes P_t, returns alpha_t and this warp's part of the block sums
+    auto softmax = [&](int t, float (&alpha)[GMAX], float (&ps)[GMAX]) -> bool {
+      const int buf = t & 1;
+      if (!warp_all(tc::mbar_wait(&c.s_full[buf], (t >> 1) & 1, abort_flag, dev_status))) return false;
+      tc::tc_fence_after();
+      uint32_t sv[16];
+      tc::tmem_ld16(tl + buf * NPAD, sv);
+      float sc[GMAX];
+#pragma unroll
+      for (int h = 0; h < GMAX; ++h) {
+        float v = h < G ? __uint_as_float(sv[h]) : -INFINITY;
+        sc[h] = v;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+        if (lane == 0 && h < G) c.rmax[buf][quarter][h] = v;
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&c.red_max);
+      if (!warp_all(tc::mbar_wait(&c.red_max, t & 1, abort_flag, dev_status))) return false;
+      uint8_t* pbase = sm + kSmemP + buf * 2 * kSmallHalf;
+#pragma unroll
+      for (int h = 0; h < GMAX; ++h) {
+        if (h < G) {
+          const float bmax = fmaxf(fmaxf(c.rmax[buf][0][h], c.rmax[buf][1][h]),
+                                   fmaxf(c.rmax[buf][2][h], c.rmax[buf][3][h]));
+          const float mn = fmaxf(m[h], bmax * a.scale_log2);
+          alpha[h] = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mn);
+          m[h] = mn;
+          const float p = ex2(fmaf(sc[h], a.scale_log2, -mn));
+          *reinterpret_cast<__nv_bfloat16*>(pbase + sw128_off(h, r, kSmallHalf)) = __float2bfloat16_rn(p);
+          ps[h] = p;
+        } else {
+          alpha[h] = 1.f;
+          ps[h] = 0.f;
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&c.p_ready[buf]);     // the MMA issuer may start PV_t
+#pragma unroll
+      for (int h = 0; h < GMAX; ++h) {
+        float v = ps[h];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        ps[h] = v;
+      }
+      return true;
+    };
+    int used = nb;
+    bool ok = true;
+    float a_cur[GMAX], p_cur[GMAX], a_nxt[GMAX], p_nxt[GMAX];
+    ok = softmax(0, a_cur, p_cur);
+    for (int t = 0; ok && t < nb; ++t) {
+      const int buf = t & 1;
+      if (t + 1 < nb) {
+        ok = softmax(t + 1, a_nxt, p_nxt);       // P_{t+1} while PV_t runs
+        if (!ok) break;
+      }
+      ok = warp_all(tc::mbar_wait(&c.o_full[buf], (t >> 1) & 1, abort_flag, dev_status));
+      if (!ok) break;
+      tc::tc_fence_after();
+      uint32_t dv[16];
+      tc::tmem_ld16(tl + 32 + buf * NPAD, dv);
+      tc::tc_fence_before();
+      if (t >= 1) {
+        // the verdict on block t-1 (usually long made): on a stop, O^(t-1) is final
+        ok = warp_all(tc::mbar_wait(&c.decided, (t - 1) & 1, abort_flag, dev_status));
+        if (!ok) break;
+        if (c.stop_at == t - 1) {
+          used = t;
+          break;
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < GMAX; ++h) {
+        if (h < G) {
+          o[h] = fmaf(o[h], a_cur[h], __uint_as_float(dv[h]));
+          lw[h] = fmaf(lw[h], a_cur[h], p_cur[h]);
+        }
+        a_cur[h] = a_nxt[h];
+        p_cur[h] = p_nxt[h];
+      }
+      c.xfull[buf][r] = o[0];
+      if (lane == 0) c.lpart[buf][quarter] = lw[0];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&c.probe_rdy);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < GMAX; ++h) c.lfin[quarter][h] = lw[h];
+    }
+    if (threadIdx.x == 64) {
+      *halt = 1;                       // nothing more to stream
+      blocks_used[bg] = ok ? used : 0;
+    }
+    // the output is written after the teardown barrier, when every warp's l part is in
+    out_ok = warp_all(ok);
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) o_fin[h] = o[h];
+  } else if (warp == 6 && lane == 0) {
+    // ---------------- decider ----------------
+    int run = 0;
+    for (int t = 0; t < nb; ++t) {
+      if (!tc::mbar_wait(&c.probe_rdy, t & 1, abort_flag, dev_status)) break;
+      const int buf = t & 1;
+      const float lt = (c.lpart[buf][0] + c.lpart[buf][1]) + (c.lpart[buf][2] + c.lpart[buf][3]);
+      double sc2 = 0.0, sp2 = 0.0, dt = 0.0;
+      for (int i = 0; i < a.n_probe; ++i) {
+        const float x = __fdiv_rn(c.xfull[buf][a.dims[i]], lt);
+        if (probe_trace) probe_trace[((size_t)bg * nb + t) * a.n_probe + i] = x;
+        const double xa = (double)x, xb = (double)c.xprev[i];
+        sc2 = __dadd_rn(sc2, __dmul_rn(xa, xa));
+        sp2 = __dadd_rn(sp2, __dmul_rn(xb, xb));
+        dt = __dadd_rn(dt, __dmul_rn(xa, xb));
+        c.xprev[i] = x;
+      }
+      bool stop = false;
+      if (t >= 1) {
+        const double nc = __dsqrt_rn(sc2), np = __dsqrt_rn(sp2);
+        const double ds = fabs(__dadd_rn(nc, -np));
+        const double den = __dmul_rn(nc, np);
+        const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
+        const bool stable = (ds < (double)a.tau) && (dd < (double)a.phi);
+        run = stable ? run + 1 : 0;
+        stop = a.enable && run >= a.patience;
+      }
+      if (stop) {
+        c.stop_at = t;
+        *halt = 1;                      // release the producer and the MMA issuer
+      }
+      tc::mbar_arrive(&c.decided);
+      if (stop) break;
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0 && lane == 0) {
+    for (int t = issued - STAGES < 0 ? 0 : issued - STAGES; t < issued; ++t)
+      tc::mbar_wait_timed(&c.kv_full[t % STAGES], (t / STAGES) & 1);
+  }
+  if (warp == 1) {
+    if (lane == 0 && mma_issued) {
+      tc::umma_commit(&c.done);
+      tc::mbar_wait_timed(&c.done, 0);
+    }
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+  if (warp >= 2 && warp <= 5 && out_ok) {
+    const int r = (warp & 3) * 32 + lane;
+    uint16_t* og = out + ((size_t)b * a.Hq + (size_t)g * G) * HD;
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < G) {
+        const float lt = (c.lfin[0][h] + c.lfin[1][h]) + (c.lfin[2][h] + c.lfin[3][h]);
+        og[h * HD + r] = f32_to_bf16_rn(lt > 0.f ? o_fin[h] / lt : 0.f);
+      }
+    }
+  }
+}
+
+bool decode_tc_supported(const bsa_decode_shape& s) {
+  const int G = s.Hq / s.Hkv;
+  return s.dtype == BSA_BF16 && s.d == HD && s.block_kv == BKV && G >= 1 && G <= GMAX &&
+         (long long)s.B * s.Hkv * s.L < (1ll << 31);
+}
+
+cudaError_t launch_decode_tc(const bsa_decode_shape& s, const DecodeArgs& a, const void* q,
+                             const void* kc, const void* vc, void* out, int32_t* blocks_used,
+                             float* probe_trace, int32_t* dev_status, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  const uint64_t rows = (uint64_t)s.B * s.Hkv * s.L;
+  if (!make_tmap_bf16_2d(&mk, kc, rows, HD, 64, BKV) || !make_tmap_bf16_2d(&mv, vc, rows, HD, 64, BKV))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  decode_tc_kernel<<<s.B * s.Hkv, kThreads, kSmemBytes, st>>>(mk, mv, (const uint16_t*)q, a,
+                                                             (uint16_t*)out, blocks_used, probe_trace,
+                                                             dev_status);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -44,7 +44,28 @@ cudaError_t launch_attend_tc(const bsa_shape& s, const void* q, const void* k, c
                              const int32_t* kv_idx, const int32_t* kv_cnt, int W, float scale,
                              void* out, float* lse, int32_t* dev_status, cudaStream_t st);
 
-// Decode with run-time termination.
+// Limits of this build (checked on the host).
+constexpr int kMaxCandidates = 8192;     // n_kb for the in-shared-memory ranking sort
+constexpr int kMaxGateTiles = 16384;     // B * n_qt for the single-CTA gate sort
+constexpr int kMaxProbe = 64;
+constexpr int kMaxGroup = 8;             // Hq / Hkv in decode
+
+// Decode kernel arguments (passed by value).
+struct DecodeArgs {
+  int L, block_kv, Hq, Hkv;
+  float scale_log2;
+  float tau, phi;
+  int patience, enable, n_probe;
+  int dims[kMaxProbe];
+};
+
+// Decode with run-time termination on tcgen05 (bf16, d 128, KV blocks of 128, Hq/Hkv <= 8).
+bool decode_tc_supported(const bsa_decode_shape& s);
+cudaError_t launch_decode_tc(const bsa_decode_shape& s, const DecodeArgs& a, const void* q,
+                             const void* kc, const void* vc, void* out, int32_t* blocks_used,
+                             float* probe_trace, int32_t* dev_status, cudaStream_t st);
+
+// Decode with run-time termination (dispatches to the tensor-core kernel where it applies).
 cudaError_t launch_decode(const bsa_decode_shape& s, const bsa_decode_params& p, const void* q,
                           const void* kc, const void* vc, float scale, void* out,
                           int32_t* blocks_used, float* probe_trace, int32_t* dev_status,
@@ -52,11 +73,5 @@ cudaError_t launch_decode(const bsa_decode_shape& s, const bsa_decode_params& p,
 
 // Sets the text bsa_last_error() returns on this thread.
 void set_last_error(const char* fmt, ...);
-
-// Limits of this build (checked on the host).
-constexpr int kMaxCandidates = 8192;     // n_kb for the in-shared-memory ranking sort
-constexpr int kMaxGateTiles = 16384;     // B * n_qt for the single-CTA gate sort
-constexpr int kMaxProbe = 64;
-constexpr int kMaxGroup = 8;             // Hq / Hkv in decode
 
 }  // namespace bsa
