@@ -63,7 +63,7 @@ struct __align__(8) Ctrl {
   float lpart[2][4];            // [block parity][warp] row-sum part of the first head
   float xfull[2][HD];           // [block parity][head dim] unnormalised O of the first head
   float lfin[4][GMAX];          // [warp][head] final row-sum parts
-  float xprev[kMaxProbe];
+  double prod[3][kMaxProbe];   // decider: per-coordinate fp64 products of the current block
 };
 
 constexpr size_t kSmemStages = 0;
@@ -318,39 +318,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     out_ok = warp_all(ok);
 #pragma unroll
     for (int h = 0; h < GMAX; ++h) o_fin[h] = o[h];
-  } else if (warp == 6 && lane == 0) {
+  } else if (warp == 6) {
     // ---------------- decider ----------------
+    // Lane i owns probe coordinates i and i + 32: it forms x = O / l for them (the
+    // fp32 divisions run in parallel), writes the trace, and the exact fp64 products
+    // x_t^2, x_{t-1}^2, x_t x_{t-1} (products of fp32 values are exact in fp64).
+    // Lane 0 adds them up in coordinate order, then tests stability.
+    const int np = a.n_probe;
+    const int d0 = lane < np ? a.dims[lane] : 0;
+    const int d1 = lane + 32 < np ? a.dims[lane + 32] : 0;
+    float xp0 = 0.f, xp1 = 0.f;
     int run = 0;
     for (int t = 0; t < nb; ++t) {
-      if (!tc::mbar_wait(&c.probe_rdy, t & 1, abort_flag, dev_status)) break;
+      if (!warp_all(tc::mbar_wait(&c.probe_rdy, t & 1, abort_flag, dev_status))) break;
       const int buf = t & 1;
       const float lt = (c.lpart[buf][0] + c.lpart[buf][1]) + (c.lpart[buf][2] + c.lpart[buf][3]);
-      double sc2 = 0.0, sp2 = 0.0, dt = 0.0;
-      for (int i = 0; i < a.n_probe; ++i) {
-        const float x = __fdiv_rn(c.xfull[buf][a.dims[i]], lt);
-        if (probe_trace) probe_trace[((size_t)bg * nb + t) * a.n_probe + i] = x;
-        const double xa = (double)x, xb = (double)c.xprev[i];
-        sc2 = __dadd_rn(sc2, __dmul_rn(xa, xa));
-        sp2 = __dadd_rn(sp2, __dmul_rn(xb, xb));
-        dt = __dadd_rn(dt, __dmul_rn(xa, xb));
-        c.xprev[i] = x;
+      const float x0 = lane < np ? __fdiv_rn(c.xfull[buf][d0], lt) : 0.f;
+      const float x1 = lane + 32 < np ? __fdiv_rn(c.xfull[buf][d1], lt) : 0.f;
+      if (probe_trace) {
+        float* tr = probe_trace + ((size_t)bg * nb + t) * np;
+        if (lane < np) tr[lane] = x0;
+        if (lane + 32 < np) tr[lane + 32] = x1;
       }
-      bool stop = false;
-      if (t >= 1) {
-        const double nc = __dsqrt_rn(sc2), np = __dsqrt_rn(sp2);
-        const double ds = fabs(__dadd_rn(nc, -np));
-        const double den = __dmul_rn(nc, np);
-        const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
-        const bool stable = (ds < (double)a.tau) && (dd < (double)a.phi);
-        run = stable ? run + 1 : 0;
-        stop = a.enable && run >= a.patience;
+      c.prod[0][lane] = __dmul_rn((double)x0, (double)x0);
+      c.prod[1][lane] = __dmul_rn((double)xp0, (double)xp0);
+      c.prod[2][lane] = __dmul_rn((double)x0, (double)xp0);
+      c.prod[0][lane + 32] = __dmul_rn((double)x1, (double)x1);
+      c.prod[1][lane + 32] = __dmul_rn((double)xp1, (double)xp1);
+      c.prod[2][lane + 32] = __dmul_rn((double)x1, (double)xp1);
+      xp0 = x0;
+      xp1 = x1;
+      __syncwarp();
+      if (lane == 0) {
+        bool stop = false;
+        if (t >= 1) {
+          double sc2 = 0.0, sp2 = 0.0, dt = 0.0;
+          for (int i = 0; i < np; ++i) {
+            sc2 = __dadd_rn(sc2, c.prod[0][i]);
+            sp2 = __dadd_rn(sp2, c.prod[1][i]);
+            dt = __dadd_rn(dt, c.prod[2][i]);
+          }
+          const double nc = __dsqrt_rn(sc2), npv = __dsqrt_rn(sp2);
+          const double ds = fabs(__dadd_rn(nc, -npv));
+          const double den = __dmul_rn(nc, npv);
+          const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
+          const bool stable = (ds < (double)a.tau) && (dd < (double)a.phi);
+          run = stable ? run + 1 : 0;
+          stop = a.enable && run >= a.patience;
+        }
+        if (stop) {
+          c.stop_at = t;
+          *halt = 1;                    // release the producer and the MMA issuer
+        }
+        tc::mbar_arrive(&c.decided);
       }
-      if (stop) {
-        c.stop_at = t;
-        *halt = 1;                      // release the producer and the MMA issuer
-      }
-      tc::mbar_arrive(&c.decided);
-      if (stop) break;
+      __syncwarp();
+      if (c.stop_at == t) break;
     }
   }
 
