@@ -6,15 +6,17 @@
 // with an online softmax. Shapes: bf16, d = 128, key blocks of 64, query
 // tiles of 128.
 //
-// One CTA per (batch, query head, query tile); 320 threads in four roles:
+// One CTA per (batch, query head, query tile); 352 threads in four roles:
 //   warp 0 (one thread)  TMA producer: the Q tile once, then K and V tiles of
 //                        128 keys = two listed blocks gathered into adjacent
 //                        shared-memory rows, two stages deep.
-//   warp 1 (one thread)  MMA issuer: S_j = Q K_j^T into one of two TMEM buffers
-//                        (S_{j+1} is issued before the value products of tile j),
-//                        then, per half tile (one listed block), O_h += P_h V_h
-//                        into that half's own TMEM accumulator as soon as the
-//                        half's P is written.
+//   warps 1, 10          MMA issuers, one thread each, one per half tile (= one
+//                        listed block): S_h = Q K_h^T (N = 64) into the half's
+//                        part of one of two TMEM S buffers (the next tile's S_h is
+//                        issued before this tile's value product), then
+//                        O_h += P_h V_h into the half's own TMEM accumulator once
+//                        the half's P is written, with P_h read straight from
+//                        tensor memory. The two halves run as separate pipelines.
 //   warps 2-9            softmax: two warps per TMEM lane quarter; a thread owns
 //                        half of one query row (the 64 keys of one listed block)
 //                        and runs an independent online softmax over the blocks
@@ -22,15 +24,19 @@
 //                        O_h accumulator, rescaled in TMEM only when its running
 //                        max grew by more than 2^8 (exact: l and O keep the same
 //                        stale max). No per-tile exchange between the halves.
+//                        P_h (bf16, two per 32-bit column) is stored with
+//                        tcgen05.st over the first 32 columns of the half's S
+//                        region, which the softmax has just read.
 //                        Epilogue: the two halves meet once, through shared
 //                        memory: m = max(m0, m1), l = l0 2^(m0-m) + l1 2^(m1-m),
 //                        O = (O_0 2^(m0-m) + O_1 2^(m1-m)) / l  -- the exact merge
 //                        of two softmax partial sums; each half writes 64 of the
 //                        128 output columns (and lse).
-// Operand layouts (all 128-byte swizzled, as TMA writes them):
-//   Q, K: K-major [rows x 64 elements] halves; P: K-major (keys are K);
-//   V: MN-major (rows = keys, 64 contiguous head dims per 128-byte row).
-// TMEM: S buffers at columns 0 and 128, O_0 at 256, O_1 at 384.
+// Shared-memory operand layouts (128-byte swizzled, as TMA writes them):
+//   Q, K: K-major [rows x 64 elements] halves; V: MN-major (rows = keys, 64
+//   contiguous head dims per 128-byte row).
+// TMEM: S buffers at columns 0 and 128 (half h at +64h; its P over the first 32
+// of those columns once read), O_0 at 256, O_1 at 384.
 // The CTA-to-work mapping walks (batch, KV head) outermost and the query heads
 // of a group innermost, so CTAs running together gather from one KV head and
 // reuse its blocks through L2.
@@ -50,7 +56,7 @@ constexpr int BQ = 128;          // query rows per tile
 constexpr int BKB = 64;          // keys per listed block
 constexpr int HD = 128;          // head dim
 constexpr int NS = 2;            // K/V pipeline stages
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kMaxList = 1024;   // kv_idx entries staged per tile
 constexpr uint32_t kHalf = 16384;            // [128 rows x 128 bytes]
@@ -63,9 +69,9 @@ constexpr uint32_t kColO = 256;              // O_0 at 256, O_1 at 384
 struct __align__(8) Ctrl {
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2], o_ready[2];   // per half tile
-  uint64_t done;
+  uint64_t s_full[2][2];                 // [half][buffer]
+  uint64_t p_full[2], o_ready[2];         // per half tile
+  uint64_t done[2];
   uint64_t lbar[4];                 // per lane quarter: both halves' (m, l) written (once)
   uint32_t tmem;
   int abort_flag;
@@ -78,8 +84,7 @@ struct __align__(8) Ctrl {
 constexpr size_t kSmemQ = 0;
 constexpr size_t kSmemK = kSmemQ + kTile;
 constexpr size_t kSmemV = kSmemK + NS * kTile;
-constexpr size_t kSmemP = kSmemV + NS * kTile;
-constexpr size_t kSmemCtrl = kSmemP + kTile;
+constexpr size_t kSmemCtrl = kSmemV + NS * kTile;
 constexpr size_t kSmemBytes = kSmemCtrl + sizeof(Ctrl) + 1024;   // + alignment slack
 
 __device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
@@ -102,7 +107,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
   const uint32_t sQ = tc::smem_u32(sm + kSmemQ);
   const uint32_t sK = tc::smem_u32(sm + kSmemK);
   const uint32_t sV = tc::smem_u32(sm + kSmemV);
-  const uint32_t sP = tc::smem_u32(sm + kSmemP);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = Hq / Hkv;
@@ -123,18 +127,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     tc::mbar_init(&c.q_full, 1);
     for (int s = 0; s < NS; ++s) {
       tc::mbar_init(&c.k_full[s], 1);
-      tc::mbar_init(&c.k_empty[s], 1);
+      tc::mbar_init(&c.k_empty[s], 2);      // both halves' S products read the K tile
       tc::mbar_init(&c.v_full[s], 1);
-      tc::mbar_init(&c.v_empty[s], 1);
+      tc::mbar_init(&c.v_empty[s], 2);      // both halves' value products read the V tile
     }
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&c.s_full[i], 1);
-      tc::mbar_init(&c.s_free[i], kSoftmaxWarps);
+      for (int bfi = 0; bfi < 2; ++bfi) tc::mbar_init(&c.s_full[i][bfi], 1);
       tc::mbar_init(&c.p_full[i], kSoftmaxWarps / 2);
       tc::mbar_init(&c.o_ready[i], 1);
+      tc::mbar_init(&c.done[i], 1);
     }
     for (int q = 0; q < 4; ++q) tc::mbar_init(&c.lbar[q], 2);
-    tc::mbar_init(&c.done, 1);
     c.abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -201,20 +204,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
       tc::tma_load_2d(vd + kHalf + kBoxK, &tmv, 64, rb, &c.v_full[s]);
       v_issued = j + 1;
     }
-  } else if (warp == 1 && lane == 0 && ntiles > 0) {
-    // ---------------- MMA issuer ----------------
-    constexpr uint32_t idS = tc::idesc_bf16_f32(128, 128, false, false);
+  } else if ((warp == 1 || warp == 10) && lane == 0 && ntiles > 0) {
+    // ---------------- MMA issuer of one half ----------------
+    const int hf = warp == 1 ? 0 : 1;
+    constexpr uint32_t idS = tc::idesc_bf16_f32(128, 64, false, false);
     constexpr uint32_t idPV = tc::idesc_bf16_f32(128, 128, false, true);
     auto issue_s = [&](int j) {
-      const uint32_t kb = sK + (j % NS) * kTile;
-      const uint32_t d = tmem + kColS + (j % 2) * 128;
+      // S_h = Q (128 x d) . K_h^T, K_h = rows 64*hf .. 64*hf+63 of the K tile
+      const uint32_t kb = sK + (j % NS) * kTile + hf * kBoxK;
+      const uint32_t d = tmem + kColS + (j % 2) * 128 + hf * 64;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
         tc::umma_bf16(d, tc::sdesc_sw128(sQ + off, 16, 1024), tc::sdesc_sw128(kb + off, 16, 1024), idS,
                       kk > 0);
       }
-      tc::umma_commit(&c.s_full[j % 2]);
+      tc::umma_commit(&c.s_full[hf][j % 2]);
       tc::umma_commit(&c.k_empty[j % NS]);
     };
     bool ok = tc::mbar_wait(&c.q_full, 0, abort_flag, dev_status) &&
@@ -227,33 +232,32 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     for (int j = 0; ok && j < ntiles; ++j) {
       const int jn = j + 1;
       if (jn < ntiles) {
+        // S_h(jn) overwrites the buffer of tile jn-2, whose P this half's value
+        // product of tile jn-2 = j-1 reads: wait for that product to complete
+        // (which also implies the softmax read S there)
         ok = tc::mbar_wait(&c.k_full[jn % NS], (jn / NS) & 1, abort_flag, dev_status) &&
-             (jn < 2 || tc::mbar_wait(&c.s_free[jn % 2], ((jn / 2) - 1) & 1, abort_flag, dev_status));
+             (jn < 2 || tc::mbar_wait(&c.o_ready[hf], (jn - 2) & 1, abort_flag, dev_status));
         if (!ok) break;
         tc::tc_fence_after();
         issue_s(jn);
       }
-      ok = tc::mbar_wait(&c.v_full[j % NS], (j / NS) & 1, abort_flag, dev_status);
+      ok = tc::mbar_wait(&c.v_full[j % NS], (j / NS) & 1, abort_flag, dev_status) &&
+           tc::mbar_wait(&c.p_full[hf], j & 1, abort_flag, dev_status);
       if (!ok) break;
+      tc::tc_fence_after();
       const uint32_t vb = sV + (j % NS) * kTile;
+      const uint32_t pa = tmem + kColS + (j % 2) * 128 + hf * 64;    // P_h in TMEM
+      // O_h += P_h (128 rows x 64 keys) . V rows of this half's block
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        ok = tc::mbar_wait(&c.p_full[half], j & 1, abort_flag, dev_status);
-        if (!ok) break;
-        tc::tc_fence_after();
-        // O_half += P_half (128 rows x 64 keys) . V rows of this half's block
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          tc::umma_bf16(tmem + kColO + half * 128, tc::sdesc_sw128(sP + half * kHalf + kk * 32, 16, 1024),
-                        tc::sdesc_sw128(vb + (half * 4 + kk) * 2048, kHalf, 1024), idPV,
-                        (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc::umma_commit(&c.o_ready[half]);
+      for (int kk = 0; kk < 4; ++kk) {
+        tc::umma_bf16_ts(tmem + kColO + hf * 128, pa + kk * 8,
+                         tc::sdesc_sw128(vb + (hf * 4 + kk) * 2048, kHalf, 1024), idPV,
+                         (j > 0 || kk > 0) ? 1u : 0u);
       }
-      if (!ok) break;
+      tc::umma_commit(&c.o_ready[hf]);
       tc::umma_commit(&c.v_empty[j % NS]);
     }
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp <= 9) {
     // ---------------- softmax warps ----------------
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;                   // 0: keys 0-63 of the tile, 1: keys 64-127
@@ -265,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     float l = 0.f;                                      // running sum of this half
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      ok = warp_all(tc::mbar_wait(&c.s_full[j % 2], (j / 2) & 1, abort_flag, dev_status));
+      ok = warp_all(tc::mbar_wait(&c.s_full[half][j % 2], (j / 2) & 1, abort_flag, dev_status));
       if (!ok) break;
       tc::tc_fence_after();
       float s[64];
@@ -276,10 +280,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(v[i]);
       }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&c.s_free[j % 2]);
-
       const bool has_b = 2 * j + 1 < nl;
       const int blk = half == 0 ? c.list[2 * j] : (has_b ? c.list[2 * j + 1] : -1);
       // mask: keys after this row, and the empty second slot of an odd tail
@@ -323,31 +323,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
       }
       l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
 
-      if (j > 0) {
-        // the previous value product of this half has read P_half and updated O_half
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // rescaling O_h: the previous value product of this half must have landed
         ok = warp_all(tc::mbar_wait(&c.o_ready[half], (j - 1) & 1, abort_flag, dev_status));
         if (!ok) break;
         tc::tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t v[32];
-            tc::tmem_ld32(tl + colO + cc * 32, v);
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          tc::tmem_ld32(tl + colO + cc * 32, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tc::tmem_st32(tl + colO + cc * 32, v);
-          }
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+          tc::tmem_st32(tl + colO + cc * 32, v);
         }
       }
-      // this half of the P row -> shared memory, 128-byte swizzle: 16-byte chunk cc of
-      // row r at cc ^ (r & 7)
-      uint8_t* prow = sm + kSmemP + half * kHalf + r * 128;
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        uint4 v4 = make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
-        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) * 16)) = v4;
-      }
-      tc::fence_proxy_async_smem();
+      // P_h -> TMEM over the first 32 columns of this half's (already read) S region
+      tc::tmem_st32(tl + kColS + (j % 2) * 128 + half * 64, pk);
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c.p_full[half]);
@@ -415,13 +406,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     for (int j = v_issued - NS < 0 ? 0 : v_issued - NS; j < v_issued; ++j)
       tc::mbar_wait_timed(&c.v_full[j % NS], (j / NS) & 1);
   }
+  if ((warp == 1 || warp == 10) && lane == 0 && mma_issued) {
+    // every MMA this thread issued has completed once this commit arrives
+    const int hf = warp == 1 ? 0 : 1;
+    tc::umma_commit(&c.done[hf]);
+    tc::mbar_wait_timed(&c.done[hf], 0);
+  }
+  __syncthreads();
   if (warp == 1) {
-    if (lane == 0 && mma_issued) {
-      // every MMA this thread issued has completed once this commit arrives
-      tc::umma_commit(&c.done);
-      tc::mbar_wait_timed(&c.done, 0);
-    }
-    __syncwarp();
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
