@@ -2,9 +2,11 @@
 // ([UGS] steps 2-5; [Stem] 2.A for the position-dependent budget).
 //
 // select_rank: one warp per (b, h, tile). The candidate blocks 0..f_lo-1 are
-//   ranked by (score desc, index asc): exact radix selection on order-preserving
-//   32-bit keys finds the m-th and M-th largest, and one pass in block order
-//   writes the top-M blocks ascending, marking the top-m ones. The cut margin
+//   ranked by (score desc, index asc): a value-bucket histogram narrows the top
+//   entries to a short list whose exact ranks come from pairwise counts within
+//   each bucket (exact radix selection on order-preserving 32-bit keys for the
+//   rows where that list is long), and the top-M blocks are written ascending,
+//   the top-m ones marked. The cut margin
 //   sigma = (s_(m-1) - s_(m)) / (s_(0) - s_(m)) is evaluated in fp32 with
 //   correctly rounded operations on the scores read back by index ([UGS] step 3).
 // gate: one CTA. sigma_bar[b,t] = fp32 sum of sigma over heads in head order,
@@ -47,10 +49,27 @@ __device__ void bitonic_sort(K* a, unsigned n, bool descending) {
 }
 
 // ---------------------------------------------------------------------------
-// Ranking: one warp per (b, h, tile) row, radix select on order-preserving
-// 32-bit keys in the warp's shared-memory slice.
+// Ranking: one warp per (b, h, tile) row; the row's scores are staged in the
+// warp's shared-memory slice.
+//
+// Bucket path. A monotone fp32 map of each score onto 256 equal-width value
+// buckets between the row's min and max (x >= y implies bucket(x) >= bucket(y),
+// since correctly rounded subtraction and multiplication are monotone) gives a
+// histogram in one pass, and from it the bucket holding the entry of rank
+// need-1, need = max(M, m+1) capped at the row length. Every entry in that bucket
+// or above is copied, in block order, to a short list; the list is regrouped by
+// bucket, and each entry's exact rank is the number of entries in higher buckets
+// plus the number in its own bucket that beat it (a greater score, or an equal
+// score at a lower block index). The ranks give the top-M list, the top-m flag
+// and the operands of sigma directly.
+//
+// Radix path, for rows the bucket path does not take (a non-finite score, all
+// scores equal, a list longer than kListCap or a bucket larger than kBucketCap):
+// exact radix selection on order-preserving 32-bit keys.
 
 constexpr uint32_t kInTopM = 0x80000000u;   // flag on a ranked entry: inside the base top-m set
+constexpr int kListCap = 256;                // longest list the bucket path takes
+constexpr uint32_t kBucketCap = 96;          // largest bucket its pairwise count takes
 
 struct RadixSel {
   uint32_t v;      // key of the element at the requested rank
@@ -124,44 +143,35 @@ __device__ __forceinline__ int warp_min_i32(int x) {
   for (int o = 16; o > 0; o >>= 1) x = min(x, __shfl_xor_sync(0xffffffffu, x, o));
   return x;
 }
+__device__ __forceinline__ float warp_min_f32(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_max_f32(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
 
-// Writes, per row, the top-M candidates (M = expanded slots) in ascending block
-// order with kInTopM set on the top-m ones (m = base slots; top-m is a prefix of
-// the same ranking, so it is a subset), and sigma from ranks 0, m-1, m.
-__global__ void __launch_bounds__(256) select_rank_kernel(
-    const float* __restrict__ scores, int rows_bh, int n_qt, int n_kb, int tile_q, int block_k,
-    int k_first, int k_last, int rho, int R, int32_t* __restrict__ ranked, float* __restrict__ sigma,
-    int32_t* dev_status) {
-  extern __shared__ uint32_t wsm[];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int wpc = blockDim.x / 32;
-  const int bh = blockIdx.y * wpc + warp;
-  if (bh >= rows_bh) return;
-  const int t = blockIdx.x;
-  uint32_t* keys = wsm + (size_t)warp * (n_kb + 256);
-  uint32_t* hist = keys + n_kb;
-  const size_t row = (size_t)bh * n_qt + t;
-  const TileSlots sl = tile_slots(t, n_qt, tile_q, block_k, k_first, k_last, rho);
-  const int n = sl.f_lo;
-  const float* s = scores + row * n_kb;
-  if (n == 0) {
-    if (lane == 0) sigma[row] = 1.0f;
-    return;
-  }
+// sigma = (s_(m-1) - s_(m)) / (s_(0) - s_(m)) with correctly rounded fp32 operations.
+__device__ __forceinline__ float cut_sigma(float s0, float a, float b) {
+  const float num = __fsub_rn(a, b);
+  const float den = __fsub_rn(s0, b);
+  return (den == 0.0f) ? 0.0f : __fdiv_rn(num, den);
+}
+
+// Radix path for one row whose keys are in keys[0..n). Writes the top-M list with
+// the top-m flag to out and returns sigma (1 when the tile has no cut).
+__device__ float rank_row_radix(const uint32_t* keys, uint32_t* hist, int n, const TileSlots& sl,
+                                const float* s, int32_t* out, int lane) {
   uint32_t kmax = 0u, kmin = 0xffffffffu;
-  bool bad = false;
   for (int i = lane; i < n; i += 32) {
-    const float x = s[i];
-    bad |= !isfinite(x);
-    const uint32_t u = score_key(x);
-    keys[i] = u;
-    kmax = max(kmax, u);
-    kmin = min(kmin, u);
+    kmax = max(kmax, keys[i]);
+    kmin = min(kmin, keys[i]);
   }
   kmax = warp_max_u32(kmax);
   kmin = warp_min_u32(kmin);
-  bad = __any_sync(0xffffffffu, bad);
-  __syncwarp();
   const int m = sl.m, M = sl.M;
   RadixSel selm{0u, 0}, selM{0u, 0};
   if (m > 0 && m < n) selm = warp_radix_select(keys, n, m - 1, kmin, kmax, hist, lane);
@@ -170,7 +180,6 @@ __global__ void __launch_bounds__(256) select_rank_kernel(
   const bool all_m = m >= n, all_M = M >= n;
 
   // one pass in block order: compaction of the top-M list, sigma bookkeeping
-  int32_t* out = ranked + row * R;
   int base_M = 0, eq_m = 0, eq_M = 0;
   int idx0 = 0x7fffffff, idx_m1 = 0x7fffffff, idx_eqnext = 0x7fffffff, idx_below = 0x7fffffff;
   uint32_t below = 0u;
@@ -205,21 +214,237 @@ __global__ void __launch_bounds__(256) select_rank_kernel(
     eq_M += __popc(bal_M);
   }
   idx0 = warp_min_i32(idx0);
-  float sg = 1.0f;
-  if (sl.cut) {
-    idx_m1 = warp_min_i32(idx_m1);
-    idx_eqnext = warp_min_i32(idx_eqnext);
-    // rank m: the next equal key if the top-m set left one out, else the best key below
-    int idx_m = idx_eqnext;
-    if (idx_m == 0x7fffffff) {
-      const uint32_t bmax = warp_max_u32(have_below ? below : 0u);
-      const bool mine = have_below && below == bmax;
-      idx_m = warp_min_i32(mine ? idx_below : 0x7fffffff);
+  if (!sl.cut) return 1.0f;
+  idx_m1 = warp_min_i32(idx_m1);
+  idx_eqnext = warp_min_i32(idx_eqnext);
+  // rank m: the next equal key if the top-m set left one out, else the best key below
+  int idx_m = idx_eqnext;
+  if (idx_m == 0x7fffffff) {
+    const uint32_t bmax = warp_max_u32(have_below ? below : 0u);
+    const bool mine = have_below && below == bmax;
+    idx_m = warp_min_i32(mine ? idx_below : 0x7fffffff);
+  }
+  return cut_sigma(s[idx0], s[idx_m1], s[idx_m]);
+}
+
+// Bin b of a 256-bin histogram lives at word (b % 8) * 32 + b / 8, so lane l's
+// eight bins 8l..8l+7 are read and written without bank conflicts.
+__device__ __forceinline__ int hidx(int b) { return ((b & 7) << 5) | (b >> 3); }
+
+struct BucketMap {
+  float lo, inv;
+  // y = (x - lo) * inv >= 0 for x >= lo; both steps are monotone, so is the bucket
+  __device__ __forceinline__ int operator()(float x) const {
+    return __float2int_rz(fminf(__fmul_rn(__fsub_rn(x, lo), inv), 255.0f));
+  }
+};
+
+__host__ __device__ inline int rank_slice_words(int n_kb) {
+  return ((n_kb + 3) & ~3) + 512 + 3 * kListCap;
+}
+
+// Writes, per row, the top-M candidates (M = expanded slots) in ascending block
+// order with kInTopM set on the top-m ones (m = base slots; top-m is a prefix of
+// the same ranking, so it is a subset), and sigma from ranks 0, m-1, m.
+__global__ void __launch_bounds__(256) select_rank_kernel(
+    const float* __restrict__ scores, int rows_bh, int n_qt, int n_kb, int tile_q, int block_k,
+    int k_first, int k_last, int rho, int R, int32_t* __restrict__ ranked, float* __restrict__ sigma,
+    int32_t* dev_status) {
+  extern __shared__ __align__(16) uint32_t wsm[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int wpc = blockDim.x / 32;
+  const int bh = blockIdx.y * wpc + warp;
+  if (bh >= rows_bh) return;
+  const int t = n_qt - 1 - (int)blockIdx.x;          // longest rows first
+  float* xs = reinterpret_cast<float*>(wsm + (size_t)warp * rank_slice_words(n_kb));
+  uint32_t* hist = reinterpret_cast<uint32_t*>(xs + ((n_kb + 3) & ~3));
+  uint32_t* start = hist + 256;
+  uint32_t* list = start + 256;                      // block index | bucket << 16, then | rank << 16
+  float* sv = reinterpret_cast<float*>(list + kListCap);   // list regrouped by bucket: scores
+  uint32_t* sp = reinterpret_cast<uint32_t*>(sv + kListCap);  // ... list position | block index << 16
+  const size_t row = (size_t)bh * n_qt + t;
+  const TileSlots sl = tile_slots(t, n_qt, tile_q, block_k, k_first, k_last, rho);
+  const int n = sl.f_lo;
+  const float* s = scores + row * n_kb;
+  int32_t* out = ranked + row * R;
+  if (n == 0) {
+    if (lane == 0) sigma[row] = 1.0f;
+    return;
+  }
+
+  // stage the row; its min, max and finiteness
+  float xmin = INFINITY, xmax = -INFINITY;
+  bool bad = false;
+  int done = 0;
+  if ((reinterpret_cast<uintptr_t>(s) & 15) == 0) {
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+    float4* x4 = reinterpret_cast<float4*>(xs);
+    const int n4 = n >> 2;
+    for (int c0 = 0; c0 < n4; c0 += 128) {           // four 16-byte loads per lane in flight
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        v[u] = c < n4 ? __ldg(s4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < n4) {
+          x4[c] = v[u];
+          xmin = fminf(fminf(xmin, v[u].x), fminf(v[u].y, fminf(v[u].z, v[u].w)));
+          xmax = fmaxf(fmaxf(xmax, v[u].x), fmaxf(v[u].y, fmaxf(v[u].z, v[u].w)));
+          bad |= !(isfinite(v[u].x) && isfinite(v[u].y) && isfinite(v[u].z) && isfinite(v[u].w));
+        }
+      }
     }
-    const float s0 = s[idx0], a = s[idx_m1], b = s[idx_m];
-    const float num = __fsub_rn(a, b);
-    const float den = __fsub_rn(s0, b);
-    sg = (den == 0.0f) ? 0.0f : __fdiv_rn(num, den);
+    done = 4 * n4;
+  }
+  for (int i = done + lane; i < n; i += 32) {
+    const float x = __ldg(s + i);
+    xs[i] = x;
+    xmin = fminf(xmin, x);
+    xmax = fmaxf(xmax, x);
+    bad |= !isfinite(x);
+  }
+  xmin = warp_min_f32(xmin);
+  xmax = warp_max_f32(xmax);
+  bad = __any_sync(0xffffffffu, bad);
+  __syncwarp();
+
+  const int m = sl.m, M = sl.M;
+  const int need = min(n, max(M, m + 1));
+  const unsigned lt = (1u << lane) - 1u;
+  const float4* x4 = reinterpret_cast<const float4*>(xs);
+  bool radix = bad || !(xmax > xmin);
+  float sg = 1.0f;
+  int L = 0, bcut = 0;
+  BucketMap bk{xmin, fminf(__fdiv_rn(256.0f, __fsub_rn(xmax, xmin)), 3.0e38f)};
+  if (!radix) {
+    // histogram of the buckets
+#pragma unroll
+    for (int k = 0; k < 8; ++k) hist[k * 32 + lane] = 0u;
+    __syncwarp();
+    for (int c = lane; 4 * c < n; c += 32) {
+      const float4 v = x4[c];
+      const int i = 4 * c;
+      atomicAdd(&hist[hidx(bk(v.x))], 1u);
+      if (i + 1 < n) atomicAdd(&hist[hidx(bk(v.y))], 1u);
+      if (i + 2 < n) atomicAdd(&hist[hidx(bk(v.z))], 1u);
+      if (i + 3 < n) atomicAdd(&hist[hidx(bk(v.w))], 1u);
+    }
+    __syncwarp();
+    uint32_t h8[8], ab[8], sum = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) { h8[k] = hist[k * 32 + lane]; sum += h8[k]; }
+    uint32_t incl = sum;                             // entries in the bins of lanes >= this lane
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+      if (lane + off < 32) incl += y;
+    }
+    uint32_t c = incl - sum;
+    int found = -1;
+    uint32_t len = 0;
+#pragma unroll
+    for (int k = 7; k >= 0; --k) {                   // ab[k]: entries in buckets above 8*lane+k
+      ab[k] = c;
+      if (ab[k] < (uint32_t)need && (uint32_t)need <= ab[k] + h8[k]) { found = lane * 8 + k; len = ab[k] + h8[k]; }
+      c += h8[k];
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, found >= 0)) - 1;
+    bcut = __shfl_sync(0xffffffffu, found, src);
+    L = (int)__shfl_sync(0xffffffffu, len, src);
+    uint32_t big = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (lane * 8 + k >= bcut) big = max(big, h8[k]);
+      start[k * 32 + lane] = ab[k];
+      hist[k * 32 + lane] = ab[k];                   // from here on: fill cursor of each bucket
+    }
+    big = warp_max_u32(big);
+    radix = L > kListCap || big > kBucketCap;
+    __syncwarp();
+  }
+  if (!radix) {
+    // the list: every entry in bucket bcut or above, in block order
+    int base = 0;
+    for (int c0 = 0; c0 < n; c0 += 128) {
+      const int i0 = c0 + 4 * lane;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i0 < n) v = x4[i0 >> 2];
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+      int bj[4], cnt = 0;
+      bool sj[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        bj[j] = bk(vv[j]);
+        sj[j] = i0 + j < n && bj[j] >= bcut;
+        cnt += sj[j] ? 1 : 0;
+      }
+      int inc = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += y;
+      }
+      int pos = base + inc - cnt;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (sj[j]) list[pos++] = (uint32_t)(i0 + j) | ((uint32_t)bj[j] << 16);
+      base += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    __syncwarp();
+    // regroup by bucket
+    for (int p = lane; p < L; p += 32) {
+      const uint32_t e = list[p];
+      const uint32_t idx = e & 0xffffu;
+      const uint32_t slot = atomicAdd(&hist[hidx((int)(e >> 16))], 1u);
+      sv[slot] = xs[idx];
+      sp[slot] = (uint32_t)p | (idx << 16);
+    }
+    __syncwarp();
+    // exact ranks: entries in higher buckets, plus those of the same bucket that beat this one
+    for (int q = lane; q < L; q += 32) {
+      const float v = sv[q];
+      const uint32_t pk = sp[q];
+      const uint32_t p = pk & 0xffffu, idx = pk >> 16;
+      const int hb = hidx((int)(list[p] >> 16));
+      const int lo = (int)start[hb], hi = (int)hist[hb];
+      int r = lo;
+      for (int u = lo; u < hi; ++u) {
+        const float w = sv[u];
+        r += (w > v || (w == v && (sp[u] >> 16) < idx)) ? 1 : 0;
+      }
+      list[p] = idx | ((uint32_t)r << 16);
+    }
+    __syncwarp();
+    // the top-M list in block order with the top-m flag; sigma's operands by rank
+    int base_M = 0, i_0 = 0x7fffffff, i_m1 = 0x7fffffff, i_m = 0x7fffffff;
+    for (int p0 = 0; p0 < L; p0 += 32) {
+      const int p = p0 + lane;
+      const bool live = p < L;
+      const uint32_t e = live ? list[p] : 0u;
+      const int idx = (int)(e & 0xffffu), r = (int)(e >> 16);
+      const bool in_M = live && r < M;
+      const unsigned bal = __ballot_sync(0xffffffffu, in_M);
+      if (in_M) out[base_M + __popc(bal & lt)] = idx | (r < m ? (int)kInTopM : 0);
+      base_M += __popc(bal);
+      if (live && r == 0) i_0 = idx;
+      if (live && r == m - 1) i_m1 = idx;
+      if (live && r == m) i_m = idx;
+    }
+    if (sl.cut) {
+      i_0 = warp_min_i32(i_0);
+      i_m1 = warp_min_i32(i_m1);
+      i_m = warp_min_i32(i_m);
+      sg = cut_sigma(xs[i_0], xs[i_m1], xs[i_m]);
+    }
+  } else {
+    uint32_t* keys = reinterpret_cast<uint32_t*>(xs);
+    for (int i = lane; i < n; i += 32) keys[i] = score_key(xs[i]);
+    __syncwarp();
+    sg = rank_row_radix(keys, hist, n, sl, s, out, lane);
   }
   if (lane == 0) {
     if (bad) {
@@ -231,8 +456,8 @@ __global__ void __launch_bounds__(256) select_rank_kernel(
 }
 
 static int rank_warps_per_cta(int n_kb) {
-  const size_t per_warp = ((size_t)n_kb + 256) * 4;
-  int w = (int)((96u * 1024u) / per_warp);
+  const size_t per_warp = (size_t)rank_slice_words(n_kb) * 4;
+  int w = (int)((112u * 1024u) / per_warp);
   return w < 1 ? 1 : (w > 8 ? 8 : w);
 }
 
@@ -241,12 +466,12 @@ cudaError_t launch_select_rank(const bsa_shape& s, const bsa_select_params& p, c
                                cudaStream_t st) {
   const int n_qt = s.N / s.tile_q, n_kb = s.N / s.block_k;
   const int wpc = rank_warps_per_cta(n_kb);
-  const size_t smem = (size_t)wpc * (n_kb + 256) * 4;
+  const size_t smem = (size_t)wpc * rank_slice_words(n_kb) * 4;
+  const int rows_bh = s.B * s.Hq;
+  dim3 grid(n_qt, (rows_bh + wpc - 1) / wpc);
   cudaError_t e = cudaFuncSetAttribute(select_rank_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int rows_bh = s.B * s.Hq;
-  dim3 grid(n_qt, (rows_bh + wpc - 1) / wpc);
   select_rank_kernel<<<grid, wpc * 32, smem, st>>>(scores, rows_bh, n_qt, n_kb, s.tile_q, s.block_k,
                                                    p.k_first, p.k_last, p.rho, R, ranked, sigma,
                                                    dev_status);
