@@ -387,20 +387,38 @@ def main_gpu(args):
     used = torch.empty(dspec.B, dspec.Hkv, dtype=torch.int32, device=dev)
     dst = torch.zeros(1, dtype=torch.int32, device=dev)
     dec = {}
-    for label, enable in (("terminated", 1), ("full_scan", 0)):
+    # visit lists: block 0 then most recent first (every block), and a selector-shaped
+    # subset of 64 blocks visited recency-first
+    lists = {}
+    for kind, keep in (("recency", 0), ("subset", 64)):
+        lh, ch = S.decode_block_lists(dspec, 2006 + 1000 * rank, kind, keep)
+        lists[kind] = (torch.from_numpy(lh).to(dev), torch.from_numpy(ch).to(dev), lh.shape[-1])
+    runs = (("terminated", 1, None), ("full_scan", 0, None), ("listed_recency", 1, "recency"),
+            ("listed_subset64", 1, "subset"))
+    for label, enable, lk in runs:
         dp = bb.DecodeParams(dspec.tau, dspec.phi, dspec.patience, enable, len(dims), cdims)
+
+        def run_decode():
+            if lk is None:
+                bb.bsa_decode(dshape, dp, dq, dk, dv, 1 / math.sqrt(dspec.d), dout, used, None, dst, sh)
+            else:
+                bl, bc, bw = lists[lk]
+                bb.bsa_decode_list(dshape, dp, dq, dk, dv, bl, bc, bw, 1 / math.sqrt(dspec.d), dout,
+                                   used, None, dst, sh)
         for _ in range(3):
-            bb.bsa_decode(dshape, dp, dq, dk, dv, 1 / math.sqrt(dspec.d), dout, used, None, dst, sh)
+            run_decode()
         torch.cuda.synchronize()
         ts = []
         for _ in range(max(3, args.steps)):
             flush.zero_()
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            bb.bsa_decode(dshape, dp, dq, dk, dv, 1 / math.sqrt(dspec.d), dout, used, None, dst, sh)
+            run_decode()
             b_.record(stream)
             ts.append((a, b_))
         torch.cuda.synchronize()
+        if int(dst.item()) != 0:
+            raise RuntimeError(f"decode {label}: device status {int(dst.item())}")
         ms = statistics.mean(a.elapsed_time(b_) for a, b_ in ts)
         blocks = int(used.sum().item())
         byts = blocks * dspec.block_kv * dspec.d * 2 * 2

@@ -30,7 +30,7 @@ BSA_SCORE_MEAN, BSA_SCORE_MEAN_VNORM = 0, 1
 EXPORTS = ("bsa_score_workspace_bytes", "bsa_score", "bsa_kv_idx_width",
            "bsa_select_workspace_bytes", "bsa_select", "bsa_attend", "bsa_decode",
            "bsa_status_string", "bsa_last_error", "bsa_select_noalloc_max_bytes",
-           "bsa_select_noalloc")
+           "bsa_select_noalloc", "bsa_selftest_wait", "bsa_decode_list")
 
 
 class BsaError(RuntimeError):
@@ -90,10 +90,15 @@ def lib() -> ctypes.CDLL:
         L.bsa_attend.restype = ctypes.c_int
         L.bsa_decode.argtypes = [dsp, dpp, vp, vp, vp, ctypes.c_float, vp, i32p, vp, i32p, vp]
         L.bsa_decode.restype = ctypes.c_int
+        L.bsa_decode_list.argtypes = [dsp, dpp, vp, vp, vp, i32p, i32p, ctypes.c_int, ctypes.c_float,
+                                      vp, i32p, vp, i32p, vp]
+        L.bsa_decode_list.restype = ctypes.c_int
         L.bsa_select_noalloc_max_bytes.argtypes = []
         L.bsa_select_noalloc_max_bytes.restype = sz
         L.bsa_select_noalloc.argtypes = [sp, pp, vp, i32p, i32p, vp, vp, vp, vp, i32p, vp]
         L.bsa_select_noalloc.restype = ctypes.c_int
+        L.bsa_selftest_wait.argtypes = [ctypes.c_int, i32p, i32p, vp]
+        L.bsa_selftest_wait.restype = ctypes.c_int
         L.bsa_status_string.argtypes = [ctypes.c_int]
         L.bsa_status_string.restype = ctypes.c_char_p
         L.bsa_last_error.argtypes = []
@@ -186,6 +191,11 @@ def bsa_select_noalloc(shape, params, scores, kv_idx, kv_cnt, sigma, sigma_bar, 
                                     _stream(stream)))
 
 
+def bsa_selftest_wait(mode, dev_status, completed, stream=None) -> None:
+    """Bounded-wait self-test: mode 0 lets a wait run out (BSA_DEV_TIMEOUT), mode 1 completes it."""
+    _check(lib().bsa_selftest_wait(int(mode), _ptr(dev_status), _ptr(completed), _stream(stream)))
+
+
 def bsa_attend(shape, q, k, v, kv_idx, kv_cnt, W, scale, out, lse, dev_status, stream=None) -> None:
     _check(lib().bsa_attend(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_idx),
                             _ptr(kv_cnt), W, scale, _ptr(out), _ptr(lse), _ptr(dev_status),
@@ -197,6 +207,14 @@ def bsa_decode(shape, params, q, k_cache, v_cache, scale, out, blocks_used, prob
     _check(lib().bsa_decode(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k_cache),
                             _ptr(v_cache), scale, _ptr(out), _ptr(blocks_used), _ptr(probe_trace),
                             _ptr(dev_status), _stream(stream)))
+
+
+def bsa_decode_list(shape, params, q, k_cache, v_cache, block_list, list_cnt, list_width, scale,
+                    out, blocks_used, probe_trace, dev_status, stream=None) -> None:
+    _check(lib().bsa_decode_list(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k_cache),
+                                 _ptr(v_cache), _ptr(block_list), _ptr(list_cnt), int(list_width),
+                                 scale, _ptr(out), _ptr(blocks_used), _ptr(probe_trace),
+                                 _ptr(dev_status), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------
@@ -254,7 +272,9 @@ def attend(q, k, v, kv_idx, kv_cnt, *, block_k: int, tile_q: int, scale: Optiona
 
 def decode(q, k_cache, v_cache, *, block_kv: int, tau: float, phi: float, patience: int = 1,
            enable: bool = True, probe_dims: Sequence[int], scale: Optional[float] = None,
-           want_trace: bool = False, stream=None):
+           want_trace: bool = False, block_list=None, list_cnt=None, stream=None):
+    """Decode with run-time termination; with block_list [B,Hkv,W] / list_cnt [B,Hkv]
+    (device int32) the listed blocks are visited in list order (bsa_decode_list)."""
     B, Hq, d = q.shape
     Hkv, L = k_cache.shape[1], k_cache.shape[2]
     shape = DecodeShape(B, Hq, Hkv, L, d, block_kv, BSA_BF16)
@@ -263,10 +283,15 @@ def decode(q, k_cache, v_cache, *, block_kv: int, tau: float, phi: float, patien
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     out = torch.empty_like(q)
     used = torch.empty(B, Hkv, dtype=torch.int32, device=q.device)
-    trace = (torch.full((B, Hkv, L // block_kv, len(probe_dims)), float("nan"),
+    steps = L // block_kv if block_list is None else block_list.shape[-1]
+    trace = (torch.full((B, Hkv, steps, len(probe_dims)), float("nan"),
                         dtype=torch.float32, device=q.device) if want_trace else None)
     st = torch.zeros(1, dtype=torch.int32, device=q.device)
-    bsa_decode(shape, params, q, k_cache, v_cache, scale, out, used, trace, st, stream)
+    if block_list is None:
+        bsa_decode(shape, params, q, k_cache, v_cache, scale, out, used, trace, st, stream)
+    else:
+        bsa_decode_list(shape, params, q, k_cache, v_cache, block_list, list_cnt,
+                        block_list.shape[-1], scale, out, used, trace, st, stream)
     return out, used, trace, st
 
 

@@ -239,9 +239,9 @@ bsa_status bsa_attend(const bsa_shape* s, const void* q, const void* k, const vo
   return ok();
 }
 
-bsa_status bsa_decode(const bsa_decode_shape* s, const bsa_decode_params* p, const void* q,
-                      const void* kc, const void* vc, float scale, void* out, int32_t* blocks_used,
-                      float* probe_trace, int32_t* dev_status, void* stream) {
+static bsa_status check_decode(const bsa_decode_shape* s, const bsa_decode_params* p, const void* q,
+                               const void* kc, const void* vc, float scale, const void* out,
+                               const int32_t* blocks_used, const int32_t* dev_status) {
   if (!s || !p) return fail(BSA_ERR_INVALID_ARG, "shape or params is NULL");
   if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->L < 1 || s->Hq % s->Hkv)
     return fail(BSA_ERR_INVALID_ARG, "bad B/Hq/Hkv/L");
@@ -263,11 +263,38 @@ bsa_status bsa_decode(const bsa_decode_shape* s, const bsa_decode_params* p, con
   if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(out))
     return fail(BSA_ERR_INVALID_ARG, "q/caches/out need 16-byte alignment");
   if (!(scale > 0.0f)) return fail(BSA_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  return BSA_OK;
+}
+
+bsa_status bsa_decode(const bsa_decode_shape* s, const bsa_decode_params* p, const void* q,
+                      const void* kc, const void* vc, float scale, void* out, int32_t* blocks_used,
+                      float* probe_trace, int32_t* dev_status, void* stream) {
+  bsa_status st = check_decode(s, p, q, kc, vc, scale, out, blocks_used, dev_status);
+  if (st != BSA_OK) return st;
   cudaStream_t cs = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
   if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
   e = bsa::launch_decode(*s, *p, q, kc, vc, scale, out, blocks_used, probe_trace, dev_status, cs);
   if (e != cudaSuccess) return cuda_fail(e, "decode");
+  return ok();
+}
+
+bsa_status bsa_decode_list(const bsa_decode_shape* s, const bsa_decode_params* p, const void* q,
+                           const void* kc, const void* vc, const int32_t* block_list,
+                           const int32_t* list_cnt, int list_width, float scale, void* out,
+                           int32_t* blocks_used, float* probe_trace, int32_t* dev_status,
+                           void* stream) {
+  bsa_status st = check_decode(s, p, q, kc, vc, scale, out, blocks_used, dev_status);
+  if (st != BSA_OK) return st;
+  if (!block_list || !list_cnt) return fail(BSA_ERR_INVALID_ARG, "NULL block_list or list_cnt");
+  if (list_width < 1 || list_width > bsa::kMaxDecodeList)
+    return fail(BSA_ERR_UNSUPPORTED, "list_width must be 1..%d", bsa::kMaxDecodeList);
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
+  e = bsa::launch_decode(*s, *p, q, kc, vc, scale, out, blocks_used, probe_trace, dev_status, cs,
+                         block_list, list_cnt, list_width);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_list");
   return ok();
 }
 

@@ -96,6 +96,29 @@ __device__ __forceinline__ void set_status(int32_t* st, int bit) {
   if (st) atomicOr(st, bit);
 }
 
+// One warp: copies the valid entries (0 <= j < n_blocks) of a decode visit list
+// lst[0..cnt) into out[] in list order and returns their number on every lane;
+// invalid entries are dropped and reported as BSA_DEV_BAD_INDEX. cnt outside
+// [0, cap] is reported too and clamped.
+__device__ inline int warp_compact_blocks(const int32_t* lst, int cnt, int cap, int n_blocks,
+                                          uint16_t* out, int32_t* dev_status, int lane) {
+  if (cnt < 0 || cnt > cap) {
+    if (lane == 0) set_status(dev_status, BSA_DEV_BAD_INDEX);
+    cnt = cnt < 0 ? 0 : cap;
+  }
+  int n = 0;
+  for (int base = 0; base < cnt; base += 32) {
+    const int i = base + lane;
+    const int j = i < cnt ? lst[i] : -1;
+    const bool valid = i < cnt && j >= 0 && j < n_blocks;
+    const unsigned m = __ballot_sync(0xffffffffu, valid);
+    if (__any_sync(0xffffffffu, i < cnt && !valid) && lane == 0) set_status(dev_status, BSA_DEV_BAD_INDEX);
+    if (valid) out[n + __popc(m & ((1u << lane) - 1u))] = (uint16_t)j;
+    n += __popc(m);
+  }
+  return n;
+}
+
 // Order-preserving map of an fp32 score to uint32 (larger score -> larger key).
 // -0.0 is folded into +0.0 so that equal scores compare equal, as IEEE does.
 __device__ __forceinline__ uint32_t score_key(float s) {

@@ -45,7 +45,7 @@ template <int D, int G>
 __global__ void __launch_bounds__(kThreads) decode_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
     const uint16_t* __restrict__ vc, const DecodeArgs a, uint16_t* __restrict__ out,
-    int32_t* __restrict__ blocks_used, float* __restrict__ probe_trace) {
+    int32_t* __restrict__ blocks_used, float* __restrict__ probe_trace, int32_t* dev_status) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   extern __shared__ __align__(16) unsigned char smraw[];
   const int BK = a.block_kv;
@@ -56,7 +56,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
   float* part = S + G * BK;                                       // [KQ][G][D]
   __shared__ float m_s[G], l_s[G], alpha_s[G];
   __shared__ float xcur[kMaxProbe], xprev[kMaxProbe];
-  __shared__ int stop_s, run_s;
+  __shared__ int stop_s, run_s, nsteps_s;
+  __shared__ uint16_t blk_s[kMaxDecodeList];     // visit list (decode over a block list)
 
   const int bg = blockIdx.x;
   const int b = bg / a.Hkv, g = bg % a.Hkv;
@@ -69,13 +70,24 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
     qs[i] = bf16_to_f32(q[((size_t)b * a.Hq + (size_t)g * G) * D + i]);
   if (tid < G) { m_s[tid] = -INFINITY; l_s[tid] = 0.f; }
   if (tid == 0) { stop_s = 0; run_s = 0; }
+  if (tid < 32) {
+    int n = nb;
+    if (a.blist)
+      n = warp_compact_blocks(a.blist + (size_t)bg * a.list_w, a.bcnt[bg], a.list_w, nb, blk_s,
+                              dev_status, tid);
+    if (tid == 0) nsteps_s = n;
+  }
+  __syncthreads();
+  const int ns = nsteps_s;                            // visit steps
+  const int tstride = a.blist ? a.list_w : nb;        // probe-trace rows per group
 
   auto issue = [&](int blk) {
-    if (blk < nb) {
+    if (blk < ns) {
       unsigned char* ks = ring + (size_t)(blk % kStages) * 2 * blk_bytes;
       unsigned char* vs = ks + blk_bytes;
-      const unsigned char* kg = reinterpret_cast<const unsigned char*>(kbase + (size_t)blk * BK * D);
-      const unsigned char* vg = reinterpret_cast<const unsigned char*>(vbase + (size_t)blk * BK * D);
+      const size_t src = a.blist ? (size_t)blk_s[blk] : (size_t)blk;
+      const unsigned char* kg = reinterpret_cast<const unsigned char*>(kbase + src * BK * D);
+      const unsigned char* vg = reinterpret_cast<const unsigned char*>(vbase + src * BK * D);
       const int chunks = BK * CPR;
       for (int c = tid; c < chunks; c += kThreads) {
         const int r = c / CPR, cc = c % CPR;
@@ -95,8 +107,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
   for (int h = 0; h < G; ++h) { acc[h][0] = 0.f; acc[h][1] = 0.f; }
 
   for (int s = 0; s < kStages - 1; ++s) issue(s);
-  int used = nb;
-  for (int blk = 0; blk < nb; ++blk) {
+  int used = ns;
+  for (int blk = 0; blk < ns; ++blk) {
     issue(blk + kStages - 1);
     cp_async_wait<kStages - 1>();
     __syncthreads();
@@ -187,7 +199,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
       for (int p = 0; p < KQ; ++p) s = __fadd_rn(s, part[p * D + dd]);
       const float x = __fdiv_rn(s, l_s[0]);
       xcur[tid] = x;
-      if (probe_trace) probe_trace[((size_t)bg * nb + blk) * a.n_probe + tid] = x;
+      if (probe_trace) probe_trace[((size_t)bg * tstride + blk) * a.n_probe + tid] = x;
     }
     __syncthreads();
     if (tid == 0) {
@@ -235,7 +247,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
 template <int D, int G>
 static cudaError_t launch_decode_t(const bsa_decode_shape& s, const DecodeArgs& a, const void* q,
                                    const void* kc, const void* vc, void* out, int32_t* blocks_used,
-                                   float* probe_trace, cudaStream_t st) {
+                                   float* probe_trace, int32_t* dev_status, cudaStream_t st) {
   const int KQ = kThreads / (D / 2);
   size_t smem = (size_t)kStages * 2 * s.block_kv * D * 2 + (size_t)G * D * 4 +
                 (size_t)G * s.block_kv * 4 + (size_t)KQ * G * D * 4;
@@ -244,30 +256,35 @@ static cudaError_t launch_decode_t(const bsa_decode_shape& s, const DecodeArgs& 
   if (e != cudaSuccess) return e;
   decode_kernel<D, G><<<s.B * s.Hkv, kThreads, smem, st>>>(
       (const uint16_t*)q, (const uint16_t*)kc, (const uint16_t*)vc, a, (uint16_t*)out, blocks_used,
-      probe_trace);
+      probe_trace, dev_status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const bsa_decode_shape& s, const bsa_decode_params& p, const void* q,
                           const void* kc, const void* vc, float scale, void* out,
                           int32_t* blocks_used, float* probe_trace, int32_t* dev_status,
-                          cudaStream_t st) {
-  // the CUDA-core kernel below has no mbarrier waits and no data-dependent indices
+                          cudaStream_t st, const int32_t* block_list, const int32_t* list_cnt,
+                          int list_w) {
+  // the CUDA-core kernel below has no mbarrier waits; its only data-dependent indices
+  // are visit-list entries, which it checks against the cache length
   DecodeArgs a;
   a.L = s.L; a.block_kv = s.block_kv; a.Hq = s.Hq; a.Hkv = s.Hkv;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.tau = p.tau; a.phi = p.phi; a.patience = p.patience; a.enable = p.enable;
   a.n_probe = p.n_probe;
   for (int i = 0; i < kMaxProbe; ++i) a.dims[i] = i < p.n_probe ? p.probe_dims[i] : 0;
+  a.blist = block_list;
+  a.bcnt = list_cnt;
+  a.list_w = block_list ? list_w : 0;
   if (decode_tc_supported(s))
     return launch_decode_tc(s, a, q, kc, vc, out, blocks_used, probe_trace, dev_status, st);
   const int G = s.Hq / s.Hkv;
 #define BSA_DEC(D)                                                                             \
   switch (G) {                                                                                 \
-    case 1: return launch_decode_t<D, 1>(s, a, q, kc, vc, out, blocks_used, probe_trace, st); \
-    case 2: return launch_decode_t<D, 2>(s, a, q, kc, vc, out, blocks_used, probe_trace, st); \
-    case 4: return launch_decode_t<D, 4>(s, a, q, kc, vc, out, blocks_used, probe_trace, st); \
-    case 8: return launch_decode_t<D, 8>(s, a, q, kc, vc, out, blocks_used, probe_trace, st); \
+    case 1: return launch_decode_t<D, 1>(s, a, q, kc, vc, out, blocks_used, probe_trace, dev_status, st); \
+    case 2: return launch_decode_t<D, 2>(s, a, q, kc, vc, out, blocks_used, probe_trace, dev_status, st); \
+    case 4: return launch_decode_t<D, 4>(s, a, q, kc, vc, out, blocks_used, probe_trace, dev_status, st); \
+    case 8: return launch_decode_t<D, 8>(s, a, q, kc, vc, out, blocks_used, probe_trace, dev_status, st); \
     default: return cudaErrorInvalidValue;                                                     \
   }
   if (s.d == 128) { BSA_DEC(128) } else { BSA_DEC(64) }

@@ -64,6 +64,8 @@ struct __align__(8) Ctrl {
   float xfull[2][HD];           // [block parity][head dim] unnormalised O of the first head
   float lfin[4][GMAX];          // [warp][head] final row-sum parts
   double prod[3][kMaxProbe];   // decider: per-coordinate fp64 products of the current block
+  int n_steps;                  // blocks to visit
+  uint16_t blk[kMaxDecodeList]; // visit list (decode over a block list)
 };
 
 constexpr size_t kSmemStages = 0;
@@ -129,6 +131,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     tc::tmem_alloc(&c.tmem, kTmemCols);
     tc::tmem_relinquish();
   }
+  if (warp == 6) {
+    int n = nb;
+    if (a.blist)
+      n = warp_compact_blocks(a.blist + (size_t)bg * a.list_w, a.bcnt[bg], a.list_w, nb, c.blk,
+                              dev_status, lane);
+    if (lane == 0) c.n_steps = n;
+  }
   if (warp >= 2 && warp <= 5) {
     // Q rows of the group (zero rows up to 16) and an all-zero P, both as K-major
     // 128-byte-swizzled MMA operands
@@ -148,6 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = c.tmem;
+  const int ns = c.n_steps;                         // visit steps
+  const int tstride = a.blist ? a.list_w : nb;      // probe-trace rows per group
   volatile int* abort_flag = &c.abort_flag;
   volatile int* halt = &c.halt;
   int issued = 0;
@@ -159,12 +170,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     // ---------------- TMA producer ----------------
     tc::prefetch_tmap(&tmk);
     tc::prefetch_tmap(&tmv);
-    for (int t = 0; t < nb; ++t) {
+    for (int t = 0; t < ns; ++t) {
       const int s = t % STAGES;
       if (t >= STAGES && !tc::mbar_wait_halt(&c.kv_empty[s], ((t / STAGES) - 1) & 1, halt, dev_status)) break;
       if (*halt) break;
       uint8_t* st = sm + kSmemStages + s * kStage;
-      const int r = row0 + t * BKV;
+      const int r = row0 + (a.blist ? (int)c.blk[t] : t) * BKV;
       tc::mbar_arrive_expect_tx(&c.kv_full[s], kStage);
       tc::tma_load_2d(st, &tmk, 0, r, &c.kv_full[s]);
       tc::tma_load_2d(st + kHalf, &tmk, 64, r, &c.kv_full[s]);
@@ -192,10 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       mma_issued = true;
       return true;
     };
-    bool ok = issue_s(0);
-    for (int t = 0; ok && t < nb; ++t) {
+    bool ok = ns > 0 && issue_s(0);
+    for (int t = 0; ok && t < ns; ++t) {
       // S_{t+1} first: its buffer held S_{t-1}, which the softmax warps read before P_{t-1}
-      if (t + 1 < nb && !issue_s(t + 1)) break;
+      if (t + 1 < ns && !issue_s(t + 1)) break;
       if (!tc::mbar_wait_halt(&c.p_ready[t & 1], (t >> 1) & 1, halt, dev_status)) break;
       tc::tc_fence_after();
       const int s = t % STAGES;
@@ -267,13 +278,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       }
       return true;
     };
-    int used = nb;
+    int used = ns;
     bool ok = true;
     float a_cur[GMAX], p_cur[GMAX], a_nxt[GMAX], p_nxt[GMAX];
-    ok = softmax(0, a_cur, p_cur);
-    for (int t = 0; ok && t < nb; ++t) {
+    if (ns > 0) ok = softmax(0, a_cur, p_cur);      // an empty visit list leaves O = 0
+    for (int t = 0; ok && t < ns; ++t) {
       const int buf = t & 1;
-      if (t + 1 < nb) {
+      if (t + 1 < ns) {
         ok = softmax(t + 1, a_nxt, p_nxt);       // P_{t+1} while PV_t runs
         if (!ok) break;
       }
@@ -329,14 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     const int d1 = lane + 32 < np ? a.dims[lane + 32] : 0;
     float xp0 = 0.f, xp1 = 0.f;
     int run = 0;
-    for (int t = 0; t < nb; ++t) {
+    for (int t = 0; t < ns; ++t) {
       if (!warp_all(tc::mbar_wait(&c.probe_rdy, t & 1, abort_flag, dev_status))) break;
       const int buf = t & 1;
       const float lt = (c.lpart[buf][0] + c.lpart[buf][1]) + (c.lpart[buf][2] + c.lpart[buf][3]);
       const float x0 = lane < np ? __fdiv_rn(c.xfull[buf][d0], lt) : 0.f;
       const float x1 = lane + 32 < np ? __fdiv_rn(c.xfull[buf][d1], lt) : 0.f;
       if (probe_trace) {
-        float* tr = probe_trace + ((size_t)bg * nb + t) * np;
+        float* tr = probe_trace + ((size_t)bg * tstride + t) * np;
         if (lane < np) tr[lane] = x0;
         if (lane + 32 < np) tr[lane + 32] = x1;
       }

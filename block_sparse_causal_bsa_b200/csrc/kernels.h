@@ -49,6 +49,7 @@ constexpr int kMaxCandidates = 8192;     // n_kb for the in-shared-memory rankin
 constexpr int kMaxGateTiles = 16384;     // B * n_qt for the single-CTA gate sort
 constexpr int kMaxProbe = 64;
 constexpr int kMaxGroup = 8;             // Hq / Hkv in decode
+constexpr int kMaxDecodeList = 4096;     // visit-list width in decode over a block list
 
 // Decode kernel arguments (passed by value).
 struct DecodeArgs {
@@ -57,6 +58,11 @@ struct DecodeArgs {
   float tau, phi;
   int patience, enable, n_probe;
   int dims[kMaxProbe];
+  // decode over a block list: blist [B, Hkv, list_w] (visit order), bcnt [B, Hkv];
+  // blist == nullptr streams blocks 0, 1, ... in order
+  const int32_t* blist;
+  const int32_t* bcnt;
+  int list_w;
 };
 
 // Decode with run-time termination on tcgen05 (bf16, d 128, KV blocks of 128, Hq/Hkv <= 8).
@@ -69,7 +75,8 @@ cudaError_t launch_decode_tc(const bsa_decode_shape& s, const DecodeArgs& a, con
 cudaError_t launch_decode(const bsa_decode_shape& s, const bsa_decode_params& p, const void* q,
                           const void* kc, const void* vc, float scale, void* out,
                           int32_t* blocks_used, float* probe_trace, int32_t* dev_status,
-                          cudaStream_t st);
+                          cudaStream_t st, const int32_t* block_list = nullptr,
+                          const int32_t* list_cnt = nullptr, int list_w = 0);
 
 // Sets the text bsa_last_error() returns on this thread.
 void set_last_error(const char* fmt, ...);

@@ -43,7 +43,7 @@ from typing import Optional
 import numpy as np
 
 _TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "vertical": 4, "latent": 5,
-               "blockmean": 6, "twin": 7, "vscale": 8}
+               "blockmean": 6, "twin": 7, "vscale": 8, "blocklist": 9}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -285,3 +285,32 @@ def default_probe_dims(n_probe: int = 32) -> np.ndarray:
     """Default probe coordinates {8m, 8m+1 : m = 0..n_probe/2-1}."""
     m = np.arange(n_probe // 2)
     return np.stack([8 * m, 8 * m + 1], axis=1).reshape(-1).astype(np.int32)
+
+
+def decode_block_lists(spec: DecodeSpec, seed: int, kind: str = "recency", keep: int = 0):
+    """Visiting orders for decode over a block list (index arithmetic only).
+
+    kind "recency": every block, block 0 first and then the most recent first
+    (n-1, n-2, ..., 1). kind "subset": block 0 first, then ``keep - 1`` other
+    blocks drawn without replacement per (batch, KV head), most recent first --
+    the shape of a selector's kv_idx visited recency-first. Returns
+    (lists [B, Hkv, W] int32 padded with -1, counts [B, Hkv] int32)."""
+    n = spec.L // spec.block_kv
+    if kind == "recency":
+        W = n
+    elif kind == "subset":
+        if not 1 <= keep <= n:
+            raise ValueError("keep must be in 1..n_blocks")
+        W = keep
+    else:
+        raise ValueError(kind)
+    lists = np.full((spec.B, spec.Hkv, W), -1, np.int32)
+    cnt = np.full((spec.B, spec.Hkv), W, np.int32)
+    for b in range(spec.B):
+        for g in range(spec.Hkv):
+            if kind == "recency":
+                lists[b, g] = np.concatenate([[0], np.arange(n - 1, 0, -1)])
+            else:
+                rest = _rng(seed, "blocklist", b, g).choice(np.arange(1, n), size=keep - 1, replace=False)
+                lists[b, g] = np.concatenate([[0], np.sort(rest)[::-1]])
+    return lists, cnt

@@ -194,6 +194,28 @@ bsa_status bsa_decode(const bsa_decode_shape* shape, const bsa_decode_params* pa
                       float softmax_scale, void* out, int32_t* blocks_used,
                       float* probe_trace, int32_t* dev_status, void* stream);
 
+/* Decode over a block list: the same stream, test and stop rule as bsa_decode, but
+ * each (batch, KV head) visits the blocks of its list in list order -- for example a
+ * selector's kv_idx visited first block first, then most important or most recent
+ * first. [ART] 2.4: a full pass does not depend on the visiting order; the first
+ * listed block is always processed (no test before the second visit step).
+ *   block_list  [B,Hkv,list_width] int32, device: block numbers (0 <= j < L/block_kv)
+ *               in visiting order; entries at or beyond list_cnt are ignored. An
+ *               out-of-range entry is skipped and reported as BSA_DEV_BAD_INDEX; a
+ *               block listed twice is visited twice (the caller lists each once).
+ *   list_cnt    [B,Hkv] int32, device: entries used (clamped to 0..list_width, with
+ *               BSA_DEV_BAD_INDEX when outside). An empty list gives out = 0,
+ *               blocks_used = 0.
+ *   list_width  1..4096 (BSA_ERR_UNSUPPORTED beyond).
+ *   blocks_used [B,Hkv] int32: visit steps processed.
+ *   probe_trace [B,Hkv,list_width,n_probe] fp32 or NULL: x^(t) per visit step.
+ * Other arguments, layouts and errors as bsa_decode. */
+bsa_status bsa_decode_list(const bsa_decode_shape* shape, const bsa_decode_params* params,
+                           const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_list, const int32_t* list_cnt, int list_width,
+                           float softmax_scale, void* out, int32_t* blocks_used,
+                           float* probe_trace, int32_t* dev_status, void* stream);
+
 /* ---- selection without a caller-provided workspace -------------------------------- */
 
 /* The pages have no counterpart to this call; it exists for callers that cannot
@@ -215,6 +237,23 @@ bsa_status bsa_select_noalloc(const bsa_shape* shape, const bsa_select_params* p
                               const float* scores, int32_t* kv_idx, int32_t* kv_cnt,
                               float* sigma, float* sigma_bar, uint8_t* trigger, float* theta,
                               int32_t* dev_status, void* stream);
+
+/* ---- self-test of the bounded device waits ------------------------------------------ */
+
+/* The pages have no counterpart to this call. It exercises, on the GPU, the bounded
+ * mbarrier wait that every tensor-core kernel of this library uses for its pipeline
+ * stages (the device-side "wait timeout" error of the calls above):
+ *   mode 0: two waits on barriers nothing completes. The first gives up after the
+ *           library's wait limit (1 s), ORs BSA_DEV_TIMEOUT into *dev_status and raises
+ *           the CTA's abort flag; the second then gives up through that flag.
+ *           completed[0] = completed[1] = 0.
+ *   mode 1: both barriers are completed first; both waits succeed, *dev_status = 0,
+ *           completed[0] = completed[1] = 1.
+ * dev_status: device int32, zeroed by the call. completed: device int32[2].
+ * Asynchronous on stream; the kernel never traps or spins without a bound, and the
+ * context stays usable afterwards. Returns BSA_ERR_INVALID_ARG for another mode or a
+ * null pointer, BSA_ERR_CUDA if the launch fails. */
+bsa_status bsa_selftest_wait(int mode, int32_t* dev_status, int32_t* completed, void* stream);
 
 /* ---- misc --------------------------------------------------------------------------- */
 

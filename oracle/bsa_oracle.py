@@ -432,3 +432,58 @@ def decode(q, Kc, Vc, block_kv, scale, tau, phi, patience, probe_dims, enable=Tr
             used[b, g] = u
             traces[b, g] = tr
     return O, used, traces
+
+
+def decode_group_list(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, block_kv: int, scale: float,
+                      blocks: Sequence[int], tau: float, phi: float, patience: int,
+                      probe_dims: np.ndarray, enable: bool = True):
+    """One (batch, KV head) visiting the listed KV blocks in list order ([ART, 2.4]:
+    the result of a full pass does not depend on the order, so a selector's blocks
+    may be visited first block first, then most important or most recent first).
+
+    After visit step t the normalised partial output O^(t) of each head is the
+    softmax over all keys of blocks[0..t] applied to V (fp64); the probe, the
+    stability test and the stop rule are those of ``decode_group`` with the visit
+    step in place of the block number (the first listed block is never tested).
+    An empty list gives O = 0 and blocks_used = 0. Returns (O [G, d] fp64,
+    blocks_used, trace [steps used, n_probe] fp32).
+    """
+    qf, Kf, Vf = widen(q), widen(Kc), widen(Vc)
+    G, d = qf.shape
+    blocks = [int(j) for j in blocks]
+    n = len(blocks)
+    if n == 0:
+        return np.zeros((G, d)), 0, np.zeros((0, len(probe_dims)), np.float32)
+    rows = np.concatenate([np.arange(j * block_kv, (j + 1) * block_kv) for j in blocks])
+    Kv, Vv = Kf[rows], Vf[rows]                        # keys in visit order
+    logits = scale * (qf @ Kv.T)                       # [G, n * block_kv]
+    e = np.exp(logits - logits.max(axis=1, keepdims=True))
+    eb = e.reshape(G, n, block_kv)
+    num = np.cumsum(np.einsum("gsk,skd->gsd", eb, Vv.reshape(n, block_kv, d)), axis=1)
+    den = np.cumsum(eb.sum(axis=2), axis=1)
+    partial = num / den[:, :, None]                    # O^(t) after each visit step
+    trace = partial[0][:, probe_dims].astype(np.float32)
+    used = termination_block(trace, tau, phi, patience) if enable else n
+    return partial[:, used - 1, :], used, trace[:used]
+
+
+def decode_list(q, Kc, Vc, block_kv, scale, block_list, list_cnt, tau, phi, patience, probe_dims,
+                enable=True):
+    """q [B,Hq,d], caches [B,Hkv,L,d], block_list [B,Hkv,W] int (visit order, the
+    first list_cnt[b,g] entries used) -> (O [B,Hq,d] fp64, blocks_used [B,Hkv],
+    traces {(b, g): trace})."""
+    B, Hq, d = q.shape
+    Hkv = Kc.shape[1]
+    G = Hq // Hkv
+    O = np.empty((B, Hq, d))
+    used = np.empty((B, Hkv), np.int32)
+    traces = {}
+    for b in range(B):
+        for g in range(Hkv):
+            lst = np.asarray(block_list[b, g][:int(list_cnt[b, g])])
+            o, u, tr = decode_group_list(q[b, g * G:(g + 1) * G], Kc[b, g], Vc[b, g], block_kv,
+                                         scale, lst, tau, phi, patience, probe_dims, enable)
+            O[b, g * G:(g + 1) * G] = o
+            used[b, g] = u
+            traces[b, g] = tr
+    return O, used, traces

@@ -458,6 +458,85 @@ def test_decode_planted_convergence():
     assert used == 2
 
 
+def test_decode_list_in_order_matches_decode():
+    """Visiting blocks 0, 1, ... through the list form gives the in-order decode."""
+    q, Kc, Vc = _decode_case()
+    dims = S.default_probe_dims(32)
+    for tau, phi in [(1e-3, 1e-4), (0.0, 0.0), (np.inf, np.inf)]:
+        a = O.decode_group(q, Kc, Vc, 128, 0.125, tau, phi, 1, dims)
+        b = O.decode_group_list(q, Kc, Vc, 128, 0.125, range(16), tau, phi, 1, dims)
+        assert a[1] == b[1]
+        np.testing.assert_allclose(a[0], b[0], rtol=0, atol=1e-13)
+        np.testing.assert_array_equal(a[2], b[2])
+
+
+def _sdpa_over_blocks(q, Kc, Vc, blocks, scale):
+    rows = np.concatenate([np.arange(j * 128, (j + 1) * 128) for j in blocks])
+    qq = torch.from_numpy(O.widen(q))[None, :, None, :]
+    kk = torch.from_numpy(O.widen(Kc)[rows])[None, None].expand(1, q.shape[0], -1, -1)
+    vv = torch.from_numpy(O.widen(Vc)[rows])[None, None].expand(1, q.shape[0], -1, -1)
+    return torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=scale)[0, :, 0].numpy()
+
+
+def test_decode_list_full_pass_is_attention_over_listed_blocks():
+    """With tau = phi = 0 nothing is stable: the output is textbook attention over
+    the keys of the listed blocks, whatever their order ([ART] 2.4)."""
+    q, Kc, Vc = _decode_case()
+    dims = S.default_probe_dims(32)
+    blocks = [0, 13, 7, 2, 9]
+    o, used, tr = O.decode_group_list(q, Kc, Vc, 128, 0.125, blocks, 0.0, 0.0, 1, dims)
+    assert used == 5 and tr.shape == (5, 32)
+    np.testing.assert_allclose(o, _sdpa_over_blocks(q, Kc, Vc, blocks, 0.125), atol=1e-12)
+    o2, _, _ = O.decode_group_list(q, Kc, Vc, 128, 0.125, [9, 2, 0, 13, 7], 0.0, 0.0, 1, dims)
+    np.testing.assert_allclose(o, o2, atol=1e-13)
+
+
+@pytest.mark.parametrize("p", [1, 3])
+def test_decode_list_infinite_thresholds(p):
+    """tau = phi = inf: every test passes, so the visit stops after p + 1 listed blocks
+    and the output is attention over exactly those."""
+    q, Kc, Vc = _decode_case()
+    blocks = [0, 15, 14, 3, 8, 1]
+    o, used, tr = O.decode_group_list(q, Kc, Vc, 128, 0.125, blocks, np.inf, np.inf, p,
+                                      S.default_probe_dims())
+    assert used == p + 1
+    np.testing.assert_allclose(o, _sdpa_over_blocks(q, Kc, Vc, blocks[:p + 1], 0.125), atol=1e-12)
+
+
+def test_decode_list_planted_first_block():
+    """The first listed block dominates (its keys align with the query): the
+    output is fixed after it, so the first test is stable and 2 steps are used."""
+    q, Kc, Vc = _decode_case()
+    qf = O.widen(q)[0]
+    Kf = np.tile(-qf, (2048, 1))
+    Kf[5 * 128:6 * 128] = 4 * qf
+    Kb = S.f32_to_bf16_bits(Kf.astype(np.float32))
+    qb = np.tile(q[0], (4, 1))
+    _, used, _ = O.decode_group_list(qb, Kb, Vc, 128, 0.125, [5, 0, 1, 2], 1e-3, 1e-4, 1,
+                                     S.default_probe_dims())
+    assert used == 2
+    _, used, _ = O.decode_group_list(qb, Kb, Vc, 128, 0.125, [0, 1, 5, 2], 1e-3, 1e-4, 1,
+                                     S.default_probe_dims())
+    assert used > 2
+
+
+def test_decode_list_empty():
+    q, Kc, Vc = _decode_case()
+    o, used, tr = O.decode_group_list(q, Kc, Vc, 128, 0.125, [], 1e-3, 1e-4, 1, S.default_probe_dims())
+    assert used == 0 and tr.shape == (0, 32) and not o.any()
+
+
+def test_decode_block_list_generator():
+    d = S.DECODE_WORKLOADS["decode_art_64k"].scaled(B=2, L=4096)
+    lists, cnt = S.decode_block_lists(d, 3, "recency")
+    assert lists.shape == (2, 8, 32) and (cnt == 32).all()
+    assert list(lists[1, 3]) == [0] + list(range(31, 0, -1))
+    lists, cnt = S.decode_block_lists(d, 3, "subset", keep=9)
+    assert lists.shape == (2, 8, 9) and (lists[:, :, 0] == 0).all()
+    for row in lists.reshape(-1, 9):
+        assert len(set(row)) == 9 and (np.diff(row[1:]) < 0).all() and row[1:].min() >= 1
+
+
 def test_generator_structure():
     """The seeded generators plant the stated structure (not method arithmetic)."""
     spec = S.WORKLOADS["gated_prefill_128k"].scaled(N=4096, Hq=4, Hkv=1)
