@@ -376,6 +376,32 @@ def main_gpu(args):
     d2h = out.numel() * 2
     del qp, kp, vp, op, qd, kd, vd, od
 
+    # the other score backbones on the same inputs (pool + score, timed on their own)
+    score_kinds = {}
+    for kind, beta in (("vnorm", 0.0), ("vlog", 0.5), ("kminmax", 0.0)):
+        code = bb.SCORE_KINDS[kind]
+        kn = bb.bsa_score_workspace_bytes(shape, code)
+        kws = torch.empty(kn, dtype=torch.uint8, device=dev)
+        kp = bb.ScoreParams(beta)
+        for _ in range(2):
+            bb.bsa_score_ex(shape, code, kp, q, k, v, scores, st_score, kws, kn, sh)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(5):
+            flush.zero_()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            bb.bsa_score_ex(shape, code, kp, q, k, v, scores, st_score, kws, kn, sh)
+            b_.record(stream)
+            ts.append((a, b_))
+        torch.cuda.synchronize()
+        if int(st_score.item()) != 0:
+            raise RuntimeError(f"score {kind}: device status {int(st_score.item())}")
+        score_kinds[kind] = {"ms": statistics.mean(a.elapsed_time(b_) for a, b_ in ts),
+                             "beta": beta if kind == "vlog" else None}
+        del kws
+    score_kinds["mean"] = {"ms": score_ms}
+
     # decode with run-time termination (timed on its own)
     dspec = S.DECODE_WORKLOADS[DECODE_WORKLOAD]
     dq, dk, dv = _gen_decode(dspec, 2005 + 1000 * rank)
@@ -457,6 +483,7 @@ def main_gpu(args):
                        "l2": "256 MB buffer written between timed steps; inputs 1.6 GB > 126 MB L2",
                        "parallelism": f"independent problem per rank x{world}"},
             "kernel_ms": {"score": score_ms, "select": select_ms, "attend": attend_ms},
+            "score_backbones_ms": score_kinds,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained,
                          "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
                          "kernel": "attend",

@@ -25,12 +25,14 @@ LIB_PATH = os.path.join(_PKG, "libbsa.so")
 BSA_OK, BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA = 0, 1, 2, 3
 BSA_DEV_OK, BSA_DEV_BAD_INDEX, BSA_DEV_TIMEOUT, BSA_DEV_BAD_SCORE = 0, 1, 2, 4
 BSA_BF16, BSA_F32 = 0, 1
-BSA_SCORE_MEAN, BSA_SCORE_MEAN_VNORM = 0, 1
+BSA_SCORE_MEAN, BSA_SCORE_MEAN_VNORM, BSA_SCORE_MEAN_VLOG, BSA_SCORE_KMINMAX = 0, 1, 2, 3
+SCORE_KINDS = {"mean": BSA_SCORE_MEAN, "vnorm": BSA_SCORE_MEAN_VNORM, "vlog": BSA_SCORE_MEAN_VLOG,
+               "kminmax": BSA_SCORE_KMINMAX}
 
 EXPORTS = ("bsa_score_workspace_bytes", "bsa_score", "bsa_kv_idx_width",
            "bsa_select_workspace_bytes", "bsa_select", "bsa_attend", "bsa_decode",
            "bsa_status_string", "bsa_last_error", "bsa_select_noalloc_max_bytes",
-           "bsa_select_noalloc", "bsa_selftest_wait", "bsa_decode_list")
+           "bsa_select_noalloc", "bsa_selftest_wait", "bsa_decode_list", "bsa_score_ex")
 
 
 class BsaError(RuntimeError):
@@ -43,6 +45,10 @@ class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
                 ("N", ctypes.c_int), ("d", ctypes.c_int), ("block_k", ctypes.c_int),
                 ("tile_q", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class ScoreParams(ctypes.Structure):
+    _fields_ = [("beta", ctypes.c_float)]
 
 
 class SelectParams(ctypes.Structure):
@@ -79,6 +85,9 @@ def lib() -> ctypes.CDLL:
         L.bsa_score_workspace_bytes.restype = sz
         L.bsa_score.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, i32p, vp, sz, vp]
         L.bsa_score.restype = ctypes.c_int
+        L.bsa_score_ex.argtypes = [sp, ctypes.c_int, ctypes.POINTER(ScoreParams), vp, vp, vp, vp, i32p,
+                                   vp, sz, vp]
+        L.bsa_score_ex.restype = ctypes.c_int
         L.bsa_kv_idx_width.argtypes = [sp, pp]
         L.bsa_kv_idx_width.restype = ctypes.c_int
         L.bsa_select_workspace_bytes.argtypes = [sp, pp]
@@ -167,6 +176,12 @@ def bsa_score(shape, kind, q, k, v, scores, dev_status, ws, ws_bytes, stream=Non
                            _ptr(dev_status), _ptr(ws), ws_bytes, _stream(stream)))
 
 
+def bsa_score_ex(shape, kind, params, q, k, v, scores, dev_status, ws, ws_bytes, stream=None) -> None:
+    _check(lib().bsa_score_ex(ctypes.byref(shape), kind, ctypes.byref(params) if params is not None else None,
+                              _ptr(q), _ptr(k), _ptr(v), _ptr(scores), _ptr(dev_status), _ptr(ws),
+                              ws_bytes, _stream(stream)))
+
+
 def bsa_kv_idx_width(shape: Shape, params: SelectParams) -> int:
     return lib().bsa_kv_idx_width(ctypes.byref(shape), ctypes.byref(params))
 
@@ -225,14 +240,20 @@ def _empty_bytes(n: int, device) -> torch.Tensor:
 
 
 def score(q, k, v=None, *, block_k: int, tile_q: int, output_aware: bool = False, stream=None,
-          status: Optional[torch.Tensor] = None):
+          status: Optional[torch.Tensor] = None, kind: Optional[str] = None, beta: float = 0.0):
+    """Block scores. kind: "mean", "vnorm" (output_aware=True), "vlog" (additive value
+    term with weight beta) or "kminmax"."""
     shape = make_shape(q, k, block_k, tile_q)
-    kind = BSA_SCORE_MEAN_VNORM if output_aware else BSA_SCORE_MEAN
+    if kind is None:
+        kind = "vnorm" if output_aware else "mean"
+    code = SCORE_KINDS[kind]
     B, Hq, N, _ = q.shape
     scores = torch.empty(B, Hq, N // tile_q, N // block_k, dtype=torch.float32, device=q.device)
-    nb = bsa_score_workspace_bytes(shape, kind)
+    nb = bsa_score_workspace_bytes(shape, code)
     ws = _empty_bytes(nb, q.device)
-    bsa_score(shape, kind, q, k, v if output_aware else None, scores, status, ws, nb, stream)
+    uses_v = kind in ("vnorm", "vlog")
+    bsa_score_ex(shape, code, ScoreParams(beta), q, k, v if uses_v else None, scores, status, ws, nb,
+                 stream)
     return scores
 
 
@@ -296,12 +317,12 @@ def decode(q, k_cache, v_cache, *, block_kv: int, tau: float, phi: float, patien
 
 
 def prefill(q, k, v, *, block_k: int, tile_q: int, cfg: SelectConfig, output_aware: bool = False,
-            scale: Optional[float] = None, stream=None):
+            scale: Optional[float] = None, stream=None, kind: Optional[str] = None, beta: float = 0.0):
     """score -> select -> attend on the current stream; returns (out, selection dict, status)."""
     shape = make_shape(q, k, block_k, tile_q)
     st_score = torch.zeros(1, dtype=torch.int32, device=q.device)
     s = score(q, k, v, block_k=block_k, tile_q=tile_q, output_aware=output_aware, stream=stream,
-              status=st_score)
+              status=st_score, kind=kind, beta=beta)
     sel = select(s, shape=shape, cfg=cfg, stream=stream)
     sel["score_status"] = st_score
     out, _, st = attend(q, k, v, sel["kv_idx"], sel["kv_cnt"], block_k=block_k, tile_q=tile_q,

@@ -64,23 +64,39 @@ bsa_status check_params(const bsa_shape* s, const bsa_select_params* p) {
 }
 
 struct ScoreWs {
-  float* kbar;
-  uint16_t* hi;
+  float* kbar;       // pooled keys, or kmin (bounds)
+  float* kbar2;      // kmax (bounds)
+  uint16_t* hi;      // bf16 split of kbar, or of mid (bounds)
   uint16_t* lo;
-  float* w;
+  uint16_t* hi2;     // bf16 split of rad (bounds)
+  uint16_t* lo2;
+  float* w;          // value-block term (output-aware kinds)
   size_t bytes;
 };
 
+bool known_kind(bsa_score_kind kind) {
+  return kind == BSA_SCORE_MEAN || kind == BSA_SCORE_MEAN_VNORM || kind == BSA_SCORE_MEAN_VLOG ||
+         kind == BSA_SCORE_KMINMAX;
+}
+
 ScoreWs score_ws(const bsa_shape& s, bsa_score_kind kind, void* base) {
   const size_t nk = (size_t)s.B * s.Hkv * (s.N / s.block_k);
+  const bool bounds = kind == BSA_SCORE_KMINMAX;
+  const bool vterm = kind == BSA_SCORE_MEAN_VNORM || kind == BSA_SCORE_MEAN_VLOG;
   ScoreWs w{};
   size_t off = 0;
   char* p = (char*)base;
   w.kbar = (float*)(p + off); off += align256(nk * s.d * 4);
   w.hi = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
   w.lo = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
-  w.w = (float*)(p + off); off += (kind == BSA_SCORE_MEAN_VNORM) ? align256(nk * 4) : 0;
-  if (kind != BSA_SCORE_MEAN_VNORM) w.w = nullptr;
+  if (bounds) {
+    w.kbar2 = (float*)(p + off); off += align256(nk * s.d * 4);
+    w.hi2 = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
+    w.lo2 = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
+  }
+  if (vterm) {
+    w.w = (float*)(p + off); off += align256(nk * 4);
+  }
   w.bytes = off;
   return w;
 }
@@ -133,19 +149,25 @@ const char* bsa_status_string(bsa_status st) {
 const char* bsa_last_error(void) { return g_err; }
 
 size_t bsa_score_workspace_bytes(const bsa_shape* s, bsa_score_kind kind) {
-  if (check_shape(s) != BSA_OK) return 0;
+  if (check_shape(s) != BSA_OK || !known_kind(kind)) return 0;
   return score_ws(*s, kind, nullptr).bytes;
 }
 
-bsa_status bsa_score(const bsa_shape* s, bsa_score_kind kind, const void* q, const void* k,
-                     const void* v, float* scores, int32_t* dev_status, void* ws, size_t ws_bytes,
-                     void* stream) {
+bsa_status bsa_score_ex(const bsa_shape* s, bsa_score_kind kind, const bsa_score_params* prm,
+                        const void* q, const void* k, const void* v, float* scores,
+                        int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
   bsa_status st = check_shape(s);
   if (st != BSA_OK) return st;
-  if (kind != BSA_SCORE_MEAN && kind != BSA_SCORE_MEAN_VNORM)
-    return fail(BSA_ERR_INVALID_ARG, "unknown score kind");
+  if (!known_kind(kind)) return fail(BSA_ERR_INVALID_ARG, "unknown score kind");
   if (!q || !k || !scores || !ws) return fail(BSA_ERR_INVALID_ARG, "NULL q, k, scores or workspace");
-  if (kind == BSA_SCORE_MEAN_VNORM && !v) return fail(BSA_ERR_INVALID_ARG, "v is NULL for VNORM");
+  const bool vterm = kind == BSA_SCORE_MEAN_VNORM || kind == BSA_SCORE_MEAN_VLOG;
+  if (vterm && !v) return fail(BSA_ERR_INVALID_ARG, "v is NULL for an output-aware score");
+  float beta = 0.f;
+  if (kind == BSA_SCORE_MEAN_VLOG) {
+    if (!prm) return fail(BSA_ERR_INVALID_ARG, "BSA_SCORE_MEAN_VLOG needs params (beta)");
+    beta = prm->beta;
+    if (!(beta >= 0.f) || !(beta < INFINITY)) return fail(BSA_ERR_INVALID_ARG, "beta must be finite and >= 0");
+  }
   if (!aligned16(q) || !aligned16(k) || (v && !aligned16(v)) || ((uintptr_t)ws & 255u))
     return fail(BSA_ERR_INVALID_ARG, "q/k/v need 16-byte and workspace 256-byte alignment");
   ScoreWs w = score_ws(*s, kind, ws);
@@ -156,18 +178,30 @@ bsa_status bsa_score(const bsa_shape* s, bsa_score_kind kind, const void* q, con
     e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
     if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
   }
-  e = bsa::launch_pool(*s, k, kind == BSA_SCORE_MEAN_VNORM ? v : nullptr, w.kbar,
-                       s->dtype == BSA_BF16 ? w.hi : nullptr, w.lo, w.w, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "pool");
-  // tensor-core path for bf16, d 128, query tiles of 128; CUDA cores otherwise
-  if (bsa::score_tc_supported(*s)) {
-    e = bsa::launch_score_tc(*s, q, w.hi, w.lo, w.w, scores, dev_status, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "score (tensor cores)");
+  const bool tc = bsa::score_tc_supported(*s);      // tensor cores for bf16, d 128, tiles of 128
+  const int wmode = kind == BSA_SCORE_MEAN_VNORM ? 1 : (kind == BSA_SCORE_MEAN_VLOG ? 2 : 0);
+  if (kind == BSA_SCORE_KMINMAX) {
+    e = bsa::launch_pool_bounds(*s, k, w.kbar, w.kbar2, tc ? w.hi : nullptr, w.lo, w.hi2, w.lo2, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "pool (bounds)");
+    e = tc ? bsa::launch_score_tc(*s, q, w.hi, w.lo, nullptr, 0, scores, dev_status, cs, w.hi2, w.lo2)
+           : bsa::launch_score_simt(*s, q, w.kbar, w.kbar2, nullptr, 0, scores, cs);
   } else {
-    e = bsa::launch_score_simt(*s, q, w.kbar, w.w, scores, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "score");
+    e = bsa::launch_pool(*s, k, vterm ? v : nullptr, w.kbar, tc ? w.hi : nullptr, w.lo, w.w, cs,
+                         kind == BSA_SCORE_MEAN_VLOG ? 1 : 0, beta);
+    if (e != cudaSuccess) return cuda_fail(e, "pool");
+    e = tc ? bsa::launch_score_tc(*s, q, w.hi, w.lo, w.w, wmode, scores, dev_status, cs)
+           : bsa::launch_score_simt(*s, q, w.kbar, nullptr, w.w, wmode, scores, cs);
   }
+  if (e != cudaSuccess) return cuda_fail(e, tc ? "score (tensor cores)" : "score");
   return ok();
+}
+
+bsa_status bsa_score(const bsa_shape* s, bsa_score_kind kind, const void* q, const void* k,
+                     const void* v, float* scores, int32_t* dev_status, void* ws, size_t ws_bytes,
+                     void* stream) {
+  if (kind == BSA_SCORE_MEAN_VLOG)
+    return fail(BSA_ERR_INVALID_ARG, "BSA_SCORE_MEAN_VLOG needs beta: use bsa_score_ex");
+  return bsa_score_ex(s, kind, nullptr, q, k, v, scores, dev_status, ws, ws_bytes, stream);
 }
 
 int bsa_kv_idx_width(const bsa_shape* s, const bsa_select_params* p) {

@@ -8,20 +8,32 @@
 
 namespace bsa {
 
-// Pooled keys (+ value-block norms). kbar fp32 [B,Hkv,n_kb,d]; kbar_hi/lo bf16 split of
-// kbar (may be null); wnorm [B,Hkv,n_kb] (only when v != null).
+// Pooled keys (+ value-block term). kbar fp32 [B,Hkv,n_kb,d]; kbar_hi/lo bf16 split of
+// kbar (may be null); wnorm [B,Hkv,n_kb] (only when v != null): ||Vbar|| (wlog 0) or
+// beta * max(0, ln ||Vbar||^2) (wlog 1).
 cudaError_t launch_pool(const bsa_shape& s, const void* k, const void* v, float* kbar,
-                        uint16_t* kbar_hi, uint16_t* kbar_lo, float* wnorm, cudaStream_t st);
+                        uint16_t* kbar_hi, uint16_t* kbar_lo, float* wnorm, cudaStream_t st,
+                        int wlog = 0, float beta = 0.f);
 
-// Block scores on CUDA cores (fp32 FMA).
+// Per-coordinate key bounds: kmin, kmax fp32 [B,Hkv,n_kb,d]; for the tensor-core score
+// (pointers may be null) the bf16 hi/lo splits of mid = (kmin+kmax)/2, rad = (kmax-kmin)/2.
+cudaError_t launch_pool_bounds(const bsa_shape& s, const void* k, float* kmin, float* kmax,
+                               uint16_t* mid_hi, uint16_t* mid_lo, uint16_t* rad_hi, uint16_t* rad_lo,
+                               cudaStream_t st);
+
+// Block scores on CUDA cores (fp32). kbar2 != null selects the bounds backbone (kbar =
+// kmin, kbar2 = kmax). wmode: 0 none, 1 times wnorm, 2 plus wnorm.
 cudaError_t launch_score_simt(const bsa_shape& s, const void* q, const float* kbar,
-                              const float* wnorm, float* scores, cudaStream_t st);
+                              const float* kbar2, const float* wnorm, int wmode, float* scores,
+                              cudaStream_t st);
 
-// Block scores on tcgen05 tensor cores (bf16 inputs, hi/lo split of the pooled keys).
+// Block scores on tcgen05 tensor cores (bf16 inputs, hi/lo split of the pooled keys;
+// with rad_hi/lo given, the bounds backbone with kbar_hi/lo = mid).
 bool score_tc_supported(const bsa_shape& s);
 cudaError_t launch_score_tc(const bsa_shape& s, const void* q, const uint16_t* kbar_hi,
-                            const uint16_t* kbar_lo, const float* wnorm, float* scores,
-                            int32_t* dev_status, cudaStream_t st);
+                            const uint16_t* kbar_lo, const float* wnorm, int wmode, float* scores,
+                            int32_t* dev_status, cudaStream_t st, const uint16_t* rad_hi = nullptr,
+                            const uint16_t* rad_lo = nullptr);
 
 // Selection: ranked candidate lists + sigma, then the gate, then kv_idx.
 cudaError_t launch_select_rank(const bsa_shape& s, const bsa_select_params& p, const float* scores,

@@ -70,8 +70,27 @@ typedef enum { BSA_BF16 = 0, BSA_F32 = 1 } bsa_dtype;
  *                         ([UGS] steps 1-2: mean-pooled keys, tile max over rows).
  *   BSA_SCORE_MEAN_VNORM  the same max times || mean(V block j) ||_2, an output-aware
  *                         weighting of the block (motivated by [Stem] 2.B: value
- *                         magnitude enters the selection metric). */
-typedef enum { BSA_SCORE_MEAN = 0, BSA_SCORE_MEAN_VNORM = 1 } bsa_score_kind;
+ *                         magnitude enters the selection metric).
+ *   BSA_SCORE_MEAN_VLOG   the same max plus beta * max(0, ln || mean(V block j) ||^2):
+ *                         [Stem] 2.B's additive Output-Aware Metric at block level, the
+ *                         block's mean value vector standing for V_j (bsa_score_ex only,
+ *                         beta from bsa_score_params).
+ *   BSA_SCORE_KMINMAX     s(t,j) = max over the tile's rows i of
+ *                         sum_c max(q_ic kmin_jc, q_ic kmax_jc), kmin/kmax the per-
+ *                         coordinate minimum/maximum of block j's keys: the K-min/K-max
+ *                         upper-bound backbone named in [UGS] Metodologia step 1. */
+typedef enum {
+  BSA_SCORE_MEAN = 0,
+  BSA_SCORE_MEAN_VNORM = 1,
+  BSA_SCORE_MEAN_VLOG = 2,
+  BSA_SCORE_KMINMAX = 3
+} bsa_score_kind;
+
+/* Extra score parameters (bsa_score_ex). beta: weight of the value term of
+ * BSA_SCORE_MEAN_VLOG (in the units of the unscaled q . k). */
+typedef struct {
+  float beta;
+} bsa_score_params;
 
 /* Prefill problem. d in {64,128}; block_k, tile_q in {64,128}; N a multiple of both. */
 typedef struct {
@@ -132,14 +151,24 @@ typedef struct {
 size_t bsa_score_workspace_bytes(const bsa_shape* shape, bsa_score_kind kind);
 
 /* scores [B,Hq,n_qt,n_kb] fp32: s(t,j) for j <= J_t, -inf for j > J_t.
- * No 1/sqrt(d) factor (a common positive factor changes neither the ranking nor sigma).
+ * No 1/sqrt(d) factor (a common positive factor changes neither the ranking nor sigma;
+ * for BSA_SCORE_MEAN_VLOG the caller's beta carries the relative weight).
  * The tile max runs over all tile_q rows, unmasked.
- * q, k: inputs of `shape->dtype`; v is read only for BSA_SCORE_MEAN_VNORM (else may be NULL).
- * dev_status: device int32 or NULL (BSA_DEV_TIMEOUT if a bounded wait ran out). */
+ * q, k: inputs of `shape->dtype`; v is read only for the output-aware kinds (VNORM, VLOG;
+ * else may be NULL).
+ * dev_status: device int32 or NULL (BSA_DEV_TIMEOUT if a bounded wait ran out).
+ * bsa_score takes every kind but BSA_SCORE_MEAN_VLOG (which needs beta: INVALID_ARG). */
 bsa_status bsa_score(const bsa_shape* shape, bsa_score_kind kind,
                      const void* q, const void* k, const void* v,
                      float* scores, int32_t* dev_status, void* workspace, size_t workspace_bytes,
                      void* stream);
+
+/* bsa_score with parameters: params may be NULL except for BSA_SCORE_MEAN_VLOG, which
+ * needs a finite beta >= 0. */
+bsa_status bsa_score_ex(const bsa_shape* shape, bsa_score_kind kind, const bsa_score_params* params,
+                        const void* q, const void* k, const void* v,
+                        float* scores, int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                        void* stream);
 
 /* ---- selection ([UGS] steps 2-5; [Stem] 2.A) -------------------------------------- */
 

@@ -144,9 +144,56 @@ def score_tile(Q_tile: np.ndarray, Kbar: np.ndarray, J: int,
     return out
 
 
+def value_log_term(V: np.ndarray, block_k: int, beta: float) -> np.ndarray:
+    """beta * max(0, ln ||mean of the block's V rows||^2): the value-magnitude term of
+    [Stem, 2.B]'s additive Output-Aware Metric, taken at block level (the block's
+    mean value vector stands for V_j). fp64; a zero mean vector gives 0."""
+    Vb = pool_keys(V, block_k)
+    e = (Vb * Vb).sum(axis=-1)
+    with np.errstate(divide="ignore"):
+        lg = np.log(e)
+    return float(beta) * np.maximum(0.0, lg)
+
+
+def key_block_bounds(K: np.ndarray, block_k: int):
+    """(kmin, kmax)[..., j, :]: per-coordinate minimum and maximum over the keys of
+    block j -- the K-min/K-max backbone named in [UGS, Metodologia] (per-coordinate
+    upper bounds, Quest style). fp64."""
+    K = widen(K)
+    *lead, N, d = K.shape
+    Kb = K.reshape(*lead, N // block_k, block_k, d)
+    return Kb.min(axis=-2), Kb.max(axis=-2)
+
+
+def score_tile_bounds(Q_tile: np.ndarray, kmin: np.ndarray, kmax: np.ndarray, J: int) -> np.ndarray:
+    """One row of K-min/K-max block scores: s(t,j) = max over the tile's rows i of
+    sum_c max(q_ic kmin_jc, q_ic kmax_jc). Each term is the largest value q_ic x
+    takes for x in [kmin_jc, kmax_jc], so the sum bounds q_i . k from above for
+    every key k of block j ([UGS, Metodologia] step 1, "limites superiores por
+    coordenada"; step 2, max over the tile's rows). fp64, returned as fp32; -inf for
+    j > J."""
+    Q = widen(Q_tile)
+    n_kb = kmin.shape[0]
+    out = np.full(n_kb, NEG_INF32, dtype=np.float32)
+    for j0 in range(0, J + 1, 32):
+        j1 = min(J + 1, j0 + 32)
+        a = Q[:, None, :] * kmin[None, j0:j1, :]
+        b = Q[:, None, :] * kmax[None, j0:j1, :]
+        out[j0:j1] = np.maximum(a, b).sum(axis=-1).max(axis=0).astype(np.float32)
+    return out
+
+
 def block_scores(Q: np.ndarray, K: np.ndarray, tile_q: int, block_k: int,
-                 V: Optional[np.ndarray] = None, Hkv: Optional[int] = None) -> np.ndarray:
-    """scores [B, Hq, n_qt, n_kb] fp32; V given -> output-aware form."""
+                 V: Optional[np.ndarray] = None, Hkv: Optional[int] = None,
+                 kind: Optional[str] = None, beta: float = 0.0) -> np.ndarray:
+    """scores [B, Hq, n_qt, n_kb] fp32.
+
+    kind "mean": tile max of q . K_bar ([UGS] steps 1-2). "vnorm" (the default when
+    V is given): that max times ||mean V_j||_2. "vlog": that max plus
+    value_log_term (the additive form of [Stem, 2.B], weight beta). "bounds": the
+    K-min/K-max score of score_tile_bounds."""
+    if kind is None:
+        kind = "vnorm" if V is not None else "mean"
     B, Hq, N, d = Q.shape
     Hkv = K.shape[1]
     G = Hq // Hkv
@@ -154,13 +201,26 @@ def block_scores(Q: np.ndarray, K: np.ndarray, tile_q: int, block_k: int,
     out = np.empty((B, Hq, n_qt, n_kb), np.float32)
     for b in range(B):
         for g in range(Hkv):
-            Kbar = pool_keys(K[b, g], block_k)
-            w = value_block_norm(V[b, g], block_k) if V is not None else None
+            if kind == "bounds":
+                kmin, kmax = key_block_bounds(K[b, g], block_k)
+            else:
+                Kbar = pool_keys(K[b, g], block_k)
+            w = value_block_norm(V[b, g], block_k) if kind == "vnorm" else None
+            add = value_log_term(V[b, g], block_k, beta) if kind == "vlog" else None
             for h in range(g * G, (g + 1) * G):
                 Qh = widen(Q[b, h])
                 for t in range(n_qt):
                     _, J = tile_blocks(t, tile_q, block_k)
-                    out[b, h, t] = score_tile(Qh[t * tile_q:(t + 1) * tile_q], Kbar, J, w)
+                    Qt = Qh[t * tile_q:(t + 1) * tile_q]
+                    if kind == "bounds":
+                        out[b, h, t] = score_tile_bounds(Qt, kmin, kmax, J)
+                    elif kind == "vlog":
+                        Qt64 = widen(Qt)
+                        row = np.full(n_kb, NEG_INF32, dtype=np.float32)
+                        row[: J + 1] = ((Qt64 @ Kbar[: J + 1].T).max(axis=0) + add[: J + 1]).astype(np.float32)
+                        out[b, h, t] = row
+                    else:
+                        out[b, h, t] = score_tile(Qt, Kbar, J, w)
     return out
 
 

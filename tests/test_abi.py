@@ -132,3 +132,60 @@ def test_decode_validation():
     p3 = bb.DecodeParams(1e-3, 1e-4, 0, 1, 2, dims)
     assert L.bsa_decode(ctypes.byref(ok_shape), ctypes.byref(p3), 16, 16, 16, 0.1, 16, 16, None, 16,
                         None) == bb.BSA_ERR_INVALID_ARG
+
+
+def test_score_kinds_validation():
+    """The added score kinds: workspace sizes, and argument errors caught before any launch."""
+    L = bb.lib()
+    s = _shape()
+    nkb = 8 * 2048
+    n_mean = bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_MEAN)
+    assert bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_MEAN_VLOG) >= n_mean + nkb * 4
+    assert bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_KMINMAX) >= 2 * n_mean
+    assert bb.bsa_score_workspace_bytes(s, 7) == 0
+    big = 1 << 34
+    # the additive form needs beta: not through bsa_score, not with NULL params
+    assert L.bsa_score(ctypes.byref(s), bb.BSA_SCORE_MEAN_VLOG, 16, 16, 16, 16, None, 256, big,
+                       None) == bb.BSA_ERR_INVALID_ARG
+    assert b"bsa_score_ex" in L.bsa_last_error()
+    assert L.bsa_score_ex(ctypes.byref(s), bb.BSA_SCORE_MEAN_VLOG, None, 16, 16, 16, 16, None, 256,
+                          big, None) == bb.BSA_ERR_INVALID_ARG
+    for beta in (-1.0, float("nan"), float("inf")):
+        p = bb.ScoreParams(beta)
+        assert L.bsa_score_ex(ctypes.byref(s), bb.BSA_SCORE_MEAN_VLOG, ctypes.byref(p), 16, 16, 16,
+                              16, None, 256, big, None) == bb.BSA_ERR_INVALID_ARG
+    p = bb.ScoreParams(0.5)
+    # V is required for the additive form, unknown kinds are rejected
+    assert L.bsa_score_ex(ctypes.byref(s), bb.BSA_SCORE_MEAN_VLOG, ctypes.byref(p), 16, 16, None, 16,
+                          None, 256, big, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_score_ex(ctypes.byref(s), 9, ctypes.byref(p), 16, 16, 16, 16, None, 256, big,
+                          None) == bb.BSA_ERR_INVALID_ARG
+    # undersized workspace for the bounds backbone
+    assert L.bsa_score_ex(ctypes.byref(s), bb.BSA_SCORE_KMINMAX, None, 16, 16, None, 16, None, 256,
+                          n_mean, None) == bb.BSA_ERR_INVALID_ARG
+    assert b"workspace" in L.bsa_last_error()
+
+
+def test_decode_list_validation():
+    L = bb.lib()
+    ds = bb.DecodeShape(2, 32, 8, 8192, 128, 128, bb.BSA_BF16)
+    dims = (ctypes.c_int * 4)(0, 1, 8, 9)
+    dp = bb.DecodeParams(1e-3, 1e-4, 1, 1, 4, dims)
+    args = (16, 16, 16)
+    # list pointers required; width within 1..4096
+    assert L.bsa_decode_list(ctypes.byref(ds), ctypes.byref(dp), *args, None, 16, 8, 0.1, 16, 16, None,
+                             16, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_decode_list(ctypes.byref(ds), ctypes.byref(dp), *args, 16, 16, 0, 0.1, 16, 16, None,
+                             16, None) == bb.BSA_ERR_UNSUPPORTED
+    assert L.bsa_decode_list(ctypes.byref(ds), ctypes.byref(dp), *args, 16, 16, 5000, 0.1, 16, 16,
+                             None, 16, None) == bb.BSA_ERR_UNSUPPORTED
+    # the decode checks still apply
+    bad = bb.DecodeParams(1e-3, 1e-4, 0, 1, 4, dims)
+    assert L.bsa_decode_list(ctypes.byref(ds), ctypes.byref(bad), *args, 16, 16, 8, 0.1, 16, 16, None,
+                             16, None) == bb.BSA_ERR_INVALID_ARG
+
+
+def test_selftest_mode_validation():
+    L = bb.lib()
+    assert L.bsa_selftest_wait(3, 16, 16, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_selftest_wait(0, None, 16, None) == bb.BSA_ERR_INVALID_ARG

@@ -458,6 +458,73 @@ def test_decode_planted_convergence():
     assert used == 2
 
 
+def _small_prefill(seed, N=512, d=16, Hq=2, Hkv=1):
+    rng = np.random.default_rng(seed)
+    Q = S.f32_to_bf16_bits(rng.standard_normal((1, Hq, N, d)).astype(np.float32))
+    K = S.f32_to_bf16_bits(rng.standard_normal((1, Hkv, N, d)).astype(np.float32))
+    V = S.f32_to_bf16_bits((rng.standard_normal((1, Hkv, N, d)) * 1.5).astype(np.float32))
+    return Q, K, V
+
+
+def test_bounds_score_is_max_over_box_corners():
+    """sum_c max(q_c kmin_c, q_c kmax_c) is the maximum of q . x over the corners of
+    the block's bounding box: brute force over all 2^d corners for d = 4."""
+    rng = np.random.default_rng(7)
+    K = S.f32_to_bf16_bits(rng.standard_normal((1, 1, 256, 4)).astype(np.float32))
+    Q = S.f32_to_bf16_bits(rng.standard_normal((1, 1, 256, 4)).astype(np.float32))
+    s = O.block_scores(Q, K, 64, 32, kind="bounds")
+    kmin, kmax = O.key_block_bounds(K[0, 0], 32)
+    corners = np.array(np.meshgrid(*[[0, 1]] * 4, indexing="ij")).reshape(4, -1).T   # [16, 4]
+    Qf = O.widen(Q[0, 0])
+    for t in range(4):
+        J = (t + 1) * 2 - 1
+        for j in range(J + 1):
+            box = np.where(corners == 1, kmax[j], kmin[j])                 # [16, 4]
+            ref = (Qf[t * 64:(t + 1) * 64] @ box.T).max()
+            assert abs(float(s[0, 0, t, j]) - ref) <= 1e-6 * max(1.0, abs(ref))
+        assert np.isneginf(s[0, 0, t, J + 1:]).all()
+
+
+def test_bounds_score_bounds_every_key_and_is_exact_for_constant_blocks():
+    Q, K, _ = _small_prefill(8)
+    s = O.block_scores(Q, K, 64, 32, kind="bounds")
+    m = O.block_scores(Q, K, 64, 32, kind="mean")
+    Qf, Kf = O.widen(Q[0, 0]), O.widen(K[0, 0])
+    for t in range(8):
+        J = 2 * t + 1
+        dots = Qf[t * 64:(t + 1) * 64] @ Kf[:(J + 1) * 32].T              # every key
+        true_max = dots.reshape(64, J + 1, 32).max(axis=(0, 2))
+        assert (s[0, 0, t, :J + 1] >= true_max.astype(np.float32) - 1e-5).all()
+        assert (s[0, 0, t, :J + 1] >= m[0, 0, t, :J + 1] - 1e-5).all()
+    # a block whose keys are all equal: the bound is the exact tile max of q . k
+    Kc = K.copy()
+    Kc[0, 0, 64:96] = Kc[0, 0, 64]
+    s2 = O.block_scores(Q, Kc, 64, 32, kind="bounds")
+    m2 = O.block_scores(Q, Kc, 64, 32, kind="mean")
+    assert s2[0, 1, 3, 2] == m2[0, 1, 3, 2]
+
+
+def test_additive_value_term_closed_forms():
+    Q, K, V = _small_prefill(9)
+    m = O.block_scores(Q, K, 64, 32, kind="mean")
+    assert np.array_equal(O.block_scores(Q, K, 64, 32, V=V, kind="vlog", beta=0.0), m)
+    # block 5: every V row equals a vector of squared norm e^2 -> ln = 2 -> term = 2 beta
+    Vc = O.widen(V).copy()
+    u = np.zeros(16)
+    u[3] = math.e
+    Vc[0, 0, 160:192] = u
+    term = O.value_log_term(Vc[0, 0], 32, 0.75)
+    assert abs(term[5] - 1.5) < 1e-12
+    # a block whose mean value vector has squared norm below 1 contributes nothing
+    Vc[0, 0, 192:224] = 0.5 * np.ones(16) / 4.0
+    assert O.value_log_term(Vc[0, 0], 32, 0.75)[6] == 0.0
+    Vc[0, 0, 224:256] = 0.0
+    assert O.value_log_term(Vc[0, 0], 32, 0.75)[7] == 0.0
+    s = O.block_scores(Q, K, 64, 32, V=Vc, kind="vlog", beta=0.75)
+    np.testing.assert_allclose(s[0, :, 3, 5], (m[0, :, 3, 5].astype(np.float64) + 1.5), rtol=1e-6)
+    assert np.array_equal(s[0, :, 3, 6], m[0, :, 3, 6]) and np.array_equal(s[0, :, 3, 7], m[0, :, 3, 7])
+
+
 def test_decode_list_in_order_matches_decode():
     """Visiting blocks 0, 1, ... through the list form gives the in-order decode."""
     q, Kc, Vc = _decode_case()
