@@ -303,6 +303,7 @@ def main_gpu(args):
     st_sel = torch.zeros(1, dtype=torch.int32, device=dev)
     st_score = torch.zeros(1, dtype=torch.int32, device=dev)
     st_att = torch.zeros(1, dtype=torch.int32, device=dev)
+    st_acc = torch.zeros(1, dtype=torch.int32, device=dev)       # OR of every timed call's status
     theta = torch.empty(1, dtype=torch.float32, device=dev)
     ws_s_n = bb.bsa_score_workspace_bytes(shape, bb.BSA_SCORE_MEAN)
     ws_s = torch.empty(ws_s_n, dtype=torch.uint8, device=dev)
@@ -344,8 +345,11 @@ def main_gpu(args):
         for i in range(args.steps):
             flush.zero_()
             step(q, k, v, out, evs[i])
+            st_acc.bitwise_or_(st_sel).bitwise_or_(st_att).bitwise_or_(st_score)   # after the events
         torch.cuda.synchronize()
         clk.mark(False)
+    if int(st_acc.item()) != 0:
+        raise RuntimeError(f"prefill step: device status {int(st_acc.item())} in a timed step")
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -387,20 +391,67 @@ def main_gpu(args):
             bb.bsa_score_ex(shape, code, kp, q, k, v, scores, st_score, kws, kn, sh)
         torch.cuda.synchronize()
         ts = []
+        st_acc.zero_()
         for _ in range(5):
             flush.zero_()
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             bb.bsa_score_ex(shape, code, kp, q, k, v, scores, st_score, kws, kn, sh)
             b_.record(stream)
+            st_acc.bitwise_or_(st_score)
             ts.append((a, b_))
         torch.cuda.synchronize()
-        if int(st_score.item()) != 0:
-            raise RuntimeError(f"score {kind}: device status {int(st_score.item())}")
+        if int(st_acc.item()) != 0:
+            raise RuntimeError(f"score {kind}: device status {int(st_acc.item())}")
         score_kinds[kind] = {"ms": statistics.mean(a.elapsed_time(b_) for a, b_ in ts),
                              "beta": beta if kind == "vlog" else None}
         del kws
     score_kinds["mean"] = {"ms": score_ms}
+
+    # vertical-slash attention on the 32k vertical-slash workload (timed on its own)
+    vspec = S.WORKLOADS["prefill_32k_vs"]
+    vq, vk, vv = (_bf16(torch, x, dev) for x in _gen_prefill(vspec, 3001 + 1000 * rank))
+    nv_, ns_ = 64, 64
+    vidx = [torch.from_numpy(x).to(dev) for x in S.vs_indices(vspec, 3002 + 1000 * rank, nv_, ns_, 32)]
+    vshape = bb.make_shape(vq, vk, 64, 128)
+    vws_n = bb.bsa_attend_vs_workspace_bytes(vshape, nv_, ns_)
+    vws = torch.empty(vws_n, dtype=torch.uint8, device=dev)
+    vout = torch.empty_like(vq)
+    vst = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def run_vs():
+        bb.bsa_attend_vs(vshape, vq, vk, vv, vidx[0], vidx[1], nv_, vidx[2], vidx[3], ns_,
+                         1 / math.sqrt(vspec.d), vout, None, vst, vws, vws_n, sh)
+    for _ in range(3):
+        run_vs()
+    torch.cuda.synchronize()
+    ts = []
+    st_acc.zero_()
+    for _ in range(max(3, min(args.steps, 10))):
+        flush.zero_()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        run_vs()
+        b_.record(stream)
+        st_acc.bitwise_or_(vst)
+        ts.append((a, b_))
+    torch.cuda.synchronize()
+    if int(st_acc.item()) != 0:
+        raise RuntimeError(f"vertical-slash attend: device status {int(st_acc.item())}")
+    vs_ms = statistics.mean(a.elapsed_time(b_) for a, b_ in ts)
+    # visited (row tile, key block) pairs: the counts the list builder wrote into the workspace
+    rows_vs = vspec.B * vspec.Hq * (vspec.N // 128)
+    words = vspec.N // 64 + 1
+    a256 = lambda x: (x + 255) // 256 * 256
+    wl = min(vspec.N // 64, nv_ + 3 * ns_)
+    off_c = 2 * a256(vspec.B * vspec.Hq * words * 8) + a256(rows_vs * wl * 4)
+    visited = int(vws[off_c:off_c + rows_vs * 4].view(torch.int32).sum().item())
+    vs_flops = 4.0 * 128 * 64 * vspec.d * visited
+    vs_res = {"workload": "prefill_32k_vs", "n_vertical": nv_, "n_slash": ns_, "n_local": 32,
+              "ms": vs_ms, "visited_block_pairs": visited,
+              "visited_fraction_of_causal": visited / (vspec.B * vspec.Hq * sum(2 * t + 2 for t in range(vspec.N // 128))),
+              "executed_tflops": vs_flops / (vs_ms * 1e-3) / 1e12}
+    del vq, vk, vv, vws, vout
 
     # decode with run-time termination (timed on its own)
     dspec = S.DECODE_WORKLOADS[DECODE_WORKLOAD]
@@ -435,16 +486,18 @@ def main_gpu(args):
             run_decode()
         torch.cuda.synchronize()
         ts = []
+        st_acc.zero_()
         for _ in range(max(3, args.steps)):
             flush.zero_()
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             run_decode()
             b_.record(stream)
+            st_acc.bitwise_or_(dst)
             ts.append((a, b_))
         torch.cuda.synchronize()
-        if int(dst.item()) != 0:
-            raise RuntimeError(f"decode {label}: device status {int(dst.item())}")
+        if int(st_acc.item()) != 0:
+            raise RuntimeError(f"decode {label}: device status {int(st_acc.item())}")
         ms = statistics.mean(a.elapsed_time(b_) for a, b_ in ts)
         blocks = int(used.sum().item())
         byts = blocks * dspec.block_kv * dspec.d * 2 * 2
@@ -484,6 +537,7 @@ def main_gpu(args):
                        "parallelism": f"independent problem per rank x{world}"},
             "kernel_ms": {"score": score_ms, "select": select_ms, "attend": attend_ms},
             "score_backbones_ms": score_kinds,
+            "vertical_slash": vs_res,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained,
                          "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
                          "kernel": "attend",

@@ -32,7 +32,8 @@ SCORE_KINDS = {"mean": BSA_SCORE_MEAN, "vnorm": BSA_SCORE_MEAN_VNORM, "vlog": BS
 EXPORTS = ("bsa_score_workspace_bytes", "bsa_score", "bsa_kv_idx_width",
            "bsa_select_workspace_bytes", "bsa_select", "bsa_attend", "bsa_decode",
            "bsa_status_string", "bsa_last_error", "bsa_select_noalloc_max_bytes",
-           "bsa_select_noalloc", "bsa_selftest_wait", "bsa_decode_list", "bsa_score_ex")
+           "bsa_select_noalloc", "bsa_selftest_wait", "bsa_decode_list", "bsa_score_ex",
+           "bsa_attend_vs_workspace_bytes", "bsa_attend_vs")
 
 
 class BsaError(RuntimeError):
@@ -106,6 +107,11 @@ def lib() -> ctypes.CDLL:
         L.bsa_select_noalloc_max_bytes.restype = sz
         L.bsa_select_noalloc.argtypes = [sp, pp, vp, i32p, i32p, vp, vp, vp, vp, i32p, vp]
         L.bsa_select_noalloc.restype = ctypes.c_int
+        L.bsa_attend_vs_workspace_bytes.argtypes = [sp, ctypes.c_int, ctypes.c_int]
+        L.bsa_attend_vs_workspace_bytes.restype = sz
+        L.bsa_attend_vs.argtypes = [sp, vp, vp, vp, i32p, i32p, ctypes.c_int, i32p, i32p, ctypes.c_int,
+                                    ctypes.c_float, vp, vp, i32p, vp, sz, vp]
+        L.bsa_attend_vs.restype = ctypes.c_int
         L.bsa_selftest_wait.argtypes = [ctypes.c_int, i32p, i32p, vp]
         L.bsa_selftest_wait.restype = ctypes.c_int
         L.bsa_status_string.argtypes = [ctypes.c_int]
@@ -206,6 +212,17 @@ def bsa_select_noalloc(shape, params, scores, kv_idx, kv_cnt, sigma, sigma_bar, 
                                     _stream(stream)))
 
 
+def bsa_attend_vs_workspace_bytes(shape: Shape, Wv: int, Ws: int) -> int:
+    return lib().bsa_attend_vs_workspace_bytes(ctypes.byref(shape), int(Wv), int(Ws))
+
+
+def bsa_attend_vs(shape, q, k, v, v_idx, v_cnt, Wv, s_off, s_cnt, Ws, scale, out, lse, dev_status, ws,
+                  ws_bytes, stream=None) -> None:
+    _check(lib().bsa_attend_vs(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(v_idx), _ptr(v_cnt),
+                               int(Wv), _ptr(s_off), _ptr(s_cnt), int(Ws), scale, _ptr(out), _ptr(lse),
+                               _ptr(dev_status), _ptr(ws), ws_bytes, _stream(stream)))
+
+
 def bsa_selftest_wait(mode, dev_status, completed, stream=None) -> None:
     """Bounded-wait self-test: mode 0 lets a wait run out (BSA_DEV_TIMEOUT), mode 1 completes it."""
     _check(lib().bsa_selftest_wait(int(mode), _ptr(dev_status), _ptr(completed), _stream(stream)))
@@ -288,6 +305,24 @@ def attend(q, k, v, kv_idx, kv_cnt, *, block_k: int, tile_q: int, scale: Optiona
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
     st = torch.zeros(1, dtype=torch.int32, device=q.device)
     bsa_attend(shape, q, k, v, kv_idx, kv_cnt, kv_idx.shape[-1], scale, out, lse, st, stream)
+    return out, lse, st
+
+
+def attend_vs(q, k, v, v_idx, v_cnt, s_off, s_cnt, *, scale: Optional[float] = None,
+              want_lse: bool = False, stream=None):
+    """Vertical-slash attention (bsa_attend_vs): v_idx [B,Hq,Wv], s_off [B,Hq,Ws] and
+    their counts [B,Hq] as device int32 tensors. Returns (out, lse or None, status)."""
+    shape = make_shape(q, k, 64, 128)
+    Wv, Ws = v_idx.shape[-1], s_off.shape[-1]
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    nb = bsa_attend_vs_workspace_bytes(shape, Wv, Ws)
+    if nb == 0:
+        raise BsaError(BSA_ERR_UNSUPPORTED, lib().bsa_last_error().decode())
+    ws = _empty_bytes(nb, q.device)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
+    st = torch.zeros(1, dtype=torch.int32, device=q.device)
+    bsa_attend_vs(shape, q, k, v, v_idx, v_cnt, Wv, s_off, s_cnt, Ws, scale, out, lse, st, ws, nb, stream)
     return out, lse, st
 
 

@@ -273,6 +273,79 @@ bsa_status bsa_attend(const bsa_shape* s, const void* q, const void* k, const vo
   return ok();
 }
 
+// ---- vertical-slash attention ----------------------------------------------------------
+
+static int vs_list_width(const bsa_shape& s, int Wv, int Ws) {
+  const long long w = (long long)Wv + 3ll * Ws;        // a slash diagonal crosses <= 3 blocks per tile
+  const int n_kb = s.N / 64;
+  return (int)(w < n_kb ? w : n_kb);
+}
+
+struct VsWs {
+  unsigned long long* vbits;
+  unsigned long long* sbits;
+  int32_t* lists;
+  int32_t* counts;
+  size_t bytes;
+};
+
+static VsWs vs_ws(const bsa_shape& s, int Wl, void* base) {
+  const size_t bh = (size_t)s.B * s.Hq;
+  const size_t words = (size_t)s.N / 64 + 1;
+  const size_t rows = bh * (s.N / s.tile_q);
+  VsWs w{};
+  size_t off = 0;
+  char* p = (char*)base;
+  w.vbits = (unsigned long long*)(p + off); off += align256(bh * words * 8);
+  w.sbits = (unsigned long long*)(p + off); off += align256(bh * words * 8);
+  w.lists = (int32_t*)(p + off); off += align256(rows * Wl * 4);
+  w.counts = (int32_t*)(p + off); off += align256(rows * 4);
+  w.bytes = off;
+  return w;
+}
+
+static bsa_status check_vs(const bsa_shape* s, int Wv, int Ws) {
+  bsa_status st = check_shape(s);
+  if (st != BSA_OK) return st;
+  if (!bsa::attend_tc_supported(*s) || (long long)s->B * s->Hq * s->N >= (1ll << 31))
+    return fail(BSA_ERR_UNSUPPORTED, "vertical-slash attention takes bf16, d 128, key blocks of 64, tiles of 128");
+  if (Wv < 1 || Ws < 1) return fail(BSA_ERR_INVALID_ARG, "Wv and Ws must be >= 1");
+  if (vs_list_width(*s, Wv, Ws) > 1024)
+    return fail(BSA_ERR_UNSUPPORTED, "min(n_kb, Wv + 3*Ws) must be <= 1024");
+  return BSA_OK;
+}
+
+size_t bsa_attend_vs_workspace_bytes(const bsa_shape* s, int Wv, int Ws) {
+  if (check_vs(s, Wv, Ws) != BSA_OK) return 0;
+  return vs_ws(*s, vs_list_width(*s, Wv, Ws), nullptr).bytes;
+}
+
+bsa_status bsa_attend_vs(const bsa_shape* s, const void* q, const void* k, const void* v,
+                         const int32_t* v_idx, const int32_t* v_cnt, int Wv, const int32_t* s_off,
+                         const int32_t* s_cnt, int Ws, float scale, void* out, float* lse,
+                         int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  bsa_status st = check_vs(s, Wv, Ws);
+  if (st != BSA_OK) return st;
+  if (!q || !k || !v || !v_idx || !v_cnt || !s_off || !s_cnt || !out || !dev_status || !ws)
+    return fail(BSA_ERR_INVALID_ARG, "NULL input, index list, count, out, dev_status or workspace");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || ((uintptr_t)ws & 255u))
+    return fail(BSA_ERR_INVALID_ARG, "q/k/v/out need 16-byte and workspace 256-byte alignment");
+  if (!(scale > 0.0f)) return fail(BSA_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  const int Wl = vs_list_width(*s, Wv, Ws);
+  VsWs w = vs_ws(*s, Wl, ws);
+  if (ws_bytes < w.bytes) return fail(BSA_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, w.bytes);
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
+  e = bsa::launch_vs_prep(*s, v_idx, v_cnt, Wv, s_off, s_cnt, Ws, Wl, w.vbits, w.sbits, w.lists, w.counts,
+                          dev_status, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "vertical-slash lists");
+  e = bsa::launch_attend_tc_vs(*s, q, k, v, w.lists, w.counts, Wl, scale, out, lse, dev_status, w.vbits,
+                               w.sbits, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "vertical-slash attend");
+  return ok();
+}
+
 static bsa_status check_decode(const bsa_decode_shape* s, const bsa_decode_params* p, const void* q,
                                const void* kc, const void* vc, float scale, const void* out,
                                const int32_t* blocks_used, const int32_t* dev_status) {

@@ -43,6 +43,11 @@
 // Every mbarrier wait is bounded (tc::mbar_wait); a timeout sets
 // BSA_DEV_TIMEOUT, the CTA unwinds, waits for its own copies and MMAs, and
 // frees its TMEM. Invalid kv_idx entries are dropped with BSA_DEV_BAD_INDEX.
+// Vertical-slash variant (VS, [VSP] B.3): the block list covers the tile's
+// vertical columns and slash diagonals, and each (row i, key j) pair is kept
+// only if j <= i and (j is a vertical column or i - j is a slash offset), read
+// from per-head bitmaps: a 64-bit word of V per key block, and a 64-bit window
+// of S (bit-reversed) for the offsets i-j of the block's keys.
 #include <math.h>
 
 #include "common.cuh"
@@ -94,13 +99,37 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// Keys j0+u (u < 64) of block blk that row i keeps under the vertical-slash rule:
+// causal (u <= i-j0) and (bit j of V, or bit i-j of S). Bitmaps have N/64+1 words.
+__device__ __forceinline__ uint64_t vs_keep(const unsigned long long* __restrict__ vrow,
+                                            const unsigned long long* __restrict__ srow, int i,
+                                            int blk) {
+  const int rel = i - blk * BKB;
+  if (rel < 0) return 0ull;
+  const uint64_t causal = rel >= 63 ? ~0ull : ((2ull << rel) - 1ull);
+  const uint64_t v = __ldg(vrow + blk) & causal;
+  // window w: bit k <-> offset base + k; key u sits on offset rel - u = base + 63 - u
+  const int base = rel - 63;
+  uint64_t w;
+  if (base >= 0) {
+    const int q = base >> 6, r = base & 63;
+    const uint64_t a = __ldg(srow + q);
+    w = r ? ((a >> r) | (__ldg(srow + q + 1) << (64 - r))) : a;
+  } else {
+    w = __ldg(srow) << (-base);                      // offsets below 0 do not exist
+  }
+  return v | __brevll(w);
+}
 }  // namespace
 
+template <bool VS>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
     const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ kv_idx,
     const int32_t* __restrict__ kv_cnt, int W, float scale_log2, uint16_t* __restrict__ out,
-    float* __restrict__ lse, int32_t* dev_status, int N, int Hq, int Hkv, int n_qt, int n_kb) {
+    float* __restrict__ lse, int32_t* dev_status, int N, int Hq, int Hkv, int n_qt, int n_kb,
+    const unsigned long long* __restrict__ vbits, const unsigned long long* __restrict__ sbits) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl& c = *reinterpret_cast<Ctrl*>(sm + kSmemCtrl);
@@ -265,6 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t colO = kColO + half * 128;
     const int row_abs = t * BQ + r;
+    const unsigned long long* vrow = VS ? vbits + bh * (size_t)(N / 64 + 1) : nullptr;
+    const unsigned long long* srow = VS ? sbits + bh * (size_t)(N / 64 + 1) : nullptr;
     float m_used = -INFINITY;                           // running max of this half, scaled log2 units
     float l = 0.f;                                      // running sum of this half
     bool ok = true;
@@ -287,7 +318,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
       float mx8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-      if (diag) {
+      if (VS) {
+        const uint64_t keep = blk < 0 ? 0ull : vs_keep(vrow, srow, row_abs, blk);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          s[i] = ((keep >> i) & 1ull) ? s[i] : -INFINITY;
+          mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+        }
+      } else if (diag) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           const bool vis = blk >= 0 && blk * BKB + i <= row_abs;
@@ -423,24 +461,43 @@ bool attend_tc_supported(const bsa_shape& s) {
   return s.dtype == BSA_BF16 && s.d == HD && s.block_k == BKB && s.tile_q == BQ;
 }
 
-cudaError_t launch_attend_tc(const bsa_shape& s, const void* q, const void* k, const void* v,
-                             const int32_t* kv_idx, const int32_t* kv_cnt, int W, float scale,
-                             void* out, float* lse, int32_t* dev_status, cudaStream_t st) {
+template <bool VS>
+static cudaError_t launch_attend_tc_t(const bsa_shape& s, const void* q, const void* k, const void* v,
+                                      const int32_t* kv_idx, const int32_t* kv_cnt, int W, float scale,
+                                      void* out, float* lse, int32_t* dev_status,
+                                      const unsigned long long* vbits,
+                                      const unsigned long long* sbits, cudaStream_t st) {
   if (W > kMaxList) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
   const uint64_t qrows = (uint64_t)s.B * s.Hq * s.N, krows = (uint64_t)s.B * s.Hkv * s.N;
   if (!make_tmap_bf16_2d(&mq, q, qrows, HD, 64, BQ) || !make_tmap_bf16_2d(&mk, k, krows, HD, 64, BKB) ||
       !make_tmap_bf16_2d(&mv, v, krows, HD, 64, BKB))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<VS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const int n_qt = s.N / BQ;
   const long long grid = (long long)s.B * s.Hq * n_qt;
-  attend_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(
+  attend_tc_kernel<VS><<<(unsigned)grid, kThreads, kSmemBytes, st>>>(
       mq, mk, mv, kv_idx, kv_cnt, W, scale * 1.4426950408889634f, (uint16_t*)out, lse, dev_status,
-      s.N, s.Hq, s.Hkv, n_qt, s.N / BKB);
+      s.N, s.Hq, s.Hkv, n_qt, s.N / BKB, vbits, sbits);
   return cudaGetLastError();
+}
+
+cudaError_t launch_attend_tc(const bsa_shape& s, const void* q, const void* k, const void* v,
+                             const int32_t* kv_idx, const int32_t* kv_cnt, int W, float scale,
+                             void* out, float* lse, int32_t* dev_status, cudaStream_t st) {
+  return launch_attend_tc_t<false>(s, q, k, v, kv_idx, kv_cnt, W, scale, out, lse, dev_status, nullptr,
+                                   nullptr, st);
+}
+
+cudaError_t launch_attend_tc_vs(const bsa_shape& s, const void* q, const void* k, const void* v,
+                                const int32_t* lists, const int32_t* counts, int W, float scale,
+                                void* out, float* lse, int32_t* dev_status,
+                                const unsigned long long* vbits, const unsigned long long* sbits,
+                                cudaStream_t st) {
+  return launch_attend_tc_t<true>(s, q, k, v, lists, counts, W, scale, out, lse, dev_status, vbits,
+                                  sbits, st);
 }
 
 }  // namespace bsa

@@ -54,7 +54,7 @@ constexpr uint32_t kTmemCols = 64;        // S[2] at 0/16, D[2] at 32/48
 struct __align__(8) Ctrl {
   uint64_t kv_full[STAGES], kv_empty[STAGES];
   uint64_t s_full[2], o_full[2];
-  uint64_t red_max, p_ready[2], probe_rdy, decided, done;
+  uint64_t red_max, p_ready[2], probe_rdy, decided, done, vote;
   uint32_t tmem;
   int abort_flag;     // error: softmax warps unwind
   int halt;           // producer / MMA stop issuing (normal stop or error)
@@ -64,6 +64,7 @@ struct __align__(8) Ctrl {
   float xfull[2][HD];           // [block parity][head dim] unnormalised O of the first head
   float lfin[4][GMAX];          // [warp][head] final row-sum parts
   double prod[3][kMaxProbe];   // decider: per-coordinate fp64 products of the current block
+  int swait[2][4];              // softmax warps' wait results for S_t, by t parity
   int n_steps;                  // blocks to visit
   uint16_t blk[kMaxDecodeList]; // visit list (decode over a block list)
 };
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       tc::mbar_init(&c.o_full[i], 1);
     }
     tc::mbar_init(&c.red_max, 4);
+    tc::mbar_init(&c.vote, 4);
     tc::mbar_init(&c.p_ready[0], 4);
     tc::mbar_init(&c.p_ready[1], 4);
     tc::mbar_init(&c.probe_rdy, 4);
@@ -229,10 +231,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     float m[GMAX], lw[GMAX], o[GMAX];
 #pragma unroll
     for (int h = 0; h < GMAX; ++h) { m[h] = -INFINITY; lw[h] = 0.f; o[h] = 0.f; }
-    // softmax of block t: writes P_t, returns alpha_t and this warp's part of the block sums
-    auto softmax = [&](int t, float (&alpha)[GMAX], float (&ps)[GMAX]) -> bool {
+    // softmax of block t: writes P_t, returns alpha_t and this warp's part of the block sums.
+    // 0: done; 1: a stop was decided before S_t arrived (the MMA issuer may never issue it:
+    // it halts once the decider stops, possibly before block t landed); 2: error.
+    auto softmax = [&](int t, float (&alpha)[GMAX], float (&ps)[GMAX]) -> int {
       const int buf = t & 1;
-      if (!warp_all(tc::mbar_wait(&c.s_full[buf], (t >> 1) & 1, abort_flag, dev_status))) return false;
+      const int w = __reduce_max_sync(0xffffffffu, (unsigned)tc::mbar_wait_or_halt(
+                                          &c.s_full[buf], (t >> 1) & 1, halt, abort_flag, dev_status));
+      // the four warps act on one verdict (one may see S_t land while another sees the halt
+      // first): each posts its result and arrives on `vote` (phase t); a warp writes slot
+      // t&1 again only after every warp arrived for t+1, i.e. read its slot-t verdicts
+      if (lane == 0) c.swait[t & 1][quarter] = w;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&c.vote);
+      if (!warp_all(tc::mbar_wait(&c.vote, t & 1, abort_flag, dev_status))) return 2;
+      const int v = max(max(c.swait[t & 1][0], c.swait[t & 1][1]), max(c.swait[t & 1][2], c.swait[t & 1][3]));
+      if (v != 0) return v;
       tc::tc_fence_after();
       uint32_t sv[16];
       tc::tmem_ld16(tl + buf * NPAD, sv);
@@ -247,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c.red_max);
-      if (!warp_all(tc::mbar_wait(&c.red_max, t & 1, abort_flag, dev_status))) return false;
+      if (!warp_all(tc::mbar_wait(&c.red_max, t & 1, abort_flag, dev_status))) return 2;
       uint8_t* pbase = sm + kSmemP + buf * 2 * kSmallHalf;
 #pragma unroll
       for (int h = 0; h < GMAX; ++h) {
@@ -276,16 +290,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
         ps[h] = v;
       }
-      return true;
+      return 0;
     };
     int used = ns;
     bool ok = true;
     float a_cur[GMAX], p_cur[GMAX], a_nxt[GMAX], p_nxt[GMAX];
-    if (ns > 0) ok = softmax(0, a_cur, p_cur);      // an empty visit list leaves O = 0
+    if (ns > 0) ok = softmax(0, a_cur, p_cur) == 0;  // an empty visit list leaves O = 0
     for (int t = 0; ok && t < ns; ++t) {
       const int buf = t & 1;
       if (t + 1 < ns) {
-        ok = softmax(t + 1, a_nxt, p_nxt);       // P_{t+1} while PV_t runs
+        const int r = softmax(t + 1, a_nxt, p_nxt);   // P_{t+1} while PV_t runs
+        if (r == 1) {
+          // halted before S_{t+1}: only a stop decided on block t-1 does that; then
+          // O^(t-1) (already folded) is the result and PV_t is not needed
+          ok = t >= 1 && warp_all(tc::mbar_wait(&c.decided, (t - 1) & 1, abort_flag, dev_status)) &&
+               c.stop_at == t - 1;
+          if (ok) used = t;
+          break;
+        }
+        ok = r == 0;
         if (!ok) break;
       }
       ok = warp_all(tc::mbar_wait(&c.o_full[buf], (t >> 1) & 1, abort_flag, dev_status));

@@ -52,6 +52,18 @@ cudaError_t launch_attend_simt(const bsa_shape& s, const void* q, const void* k,
 
 // Sparse attend on tcgen05 tensor cores (bf16, d = 128, block_k = 64, tile_q = 128).
 bool attend_tc_supported(const bsa_shape& s);
+
+// Vertical-slash: bitmaps V and S per (b, h) (N/64+1 words each) and the per-tile key-block
+// lists (width Wl, ascending, -1 padded) with their counts; then the masked tensor-core attend.
+cudaError_t launch_vs_prep(const bsa_shape& s, const int32_t* v_idx, const int32_t* v_cnt, int Wv,
+                           const int32_t* s_off, const int32_t* s_cnt, int Ws, int Wl,
+                           unsigned long long* vbits, unsigned long long* sbits, int32_t* lists,
+                           int32_t* counts, int32_t* dev_status, cudaStream_t st);
+cudaError_t launch_attend_tc_vs(const bsa_shape& s, const void* q, const void* k, const void* v,
+                                const int32_t* lists, const int32_t* counts, int W, float scale,
+                                void* out, float* lse, int32_t* dev_status,
+                                const unsigned long long* vbits, const unsigned long long* sbits,
+                                cudaStream_t st);
 cudaError_t launch_attend_tc(const bsa_shape& s, const void* q, const void* k, const void* v,
                              const int32_t* kv_idx, const int32_t* kv_cnt, int W, float scale,
                              void* out, float* lse, int32_t* dev_status, cudaStream_t st);

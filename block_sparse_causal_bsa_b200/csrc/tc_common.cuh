@@ -94,6 +94,27 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return ok != 0;
 }
 
+// Wait for a phase that an early stop may leave incomplete forever. Returns 0 when the
+// phase completed, 1 when *halt was raised first, 2 when the CTA aborts (abort flag) or
+// kTimeoutNs elapse (then BSA_DEV_TIMEOUT is set and the abort flag raised).
+__device__ __forceinline__ int mbar_wait_or_halt(uint64_t* bar, uint32_t parity, volatile int* halt,
+                                                 volatile int* abort_flag, int32_t* dev_status) {
+  if (mbar_try_wait(bar, parity)) return 0;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return 0;
+    if (*halt) return 1;
+    if ((it & 127u) == 0u) {
+      if (*abort_flag) return 2;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        *abort_flag = 1;
+        set_status(dev_status, BSA_DEV_TIMEOUT);
+        return 2;
+      }
+    }
+  }
+}
+
 // Like mbar_wait, but polls the halt flag on every try: used where a normal early stop
 // (not only an error) must release the waiting thread promptly.
 __device__ __forceinline__ bool mbar_wait_halt(uint64_t* bar, uint32_t parity, volatile int* halt,

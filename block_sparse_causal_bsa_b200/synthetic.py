@@ -43,7 +43,7 @@ from typing import Optional
 import numpy as np
 
 _TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "vertical": 4, "latent": 5,
-               "blockmean": 6, "twin": 7, "vscale": 8, "blocklist": 9}
+               "blockmean": 6, "twin": 7, "vscale": 8, "blocklist": 9, "vsidx": 10}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -314,3 +314,32 @@ def decode_block_lists(spec: DecodeSpec, seed: int, kind: str = "recency", keep:
                 rest = _rng(seed, "blocklist", b, g).choice(np.arange(1, n), size=keep - 1, replace=False)
                 lists[b, g] = np.concatenate([[0], np.sort(rest)[::-1]])
     return lists, cnt
+
+
+def vs_indices(spec: PrefillSpec, seed: int, n_vertical: int = 64, n_slash: int = 64,
+               n_local: int = 32):
+    """Vertical and slash indices per (batch, query head) shaped like a vertical-slash
+    indexer's output (index arithmetic only): the vertical columns are the KV head's
+    planted anchor positions (the "vertical_slash" structure), the first 4 positions,
+    and seeded random positions, n_vertical in all; the slash offsets are the local
+    band 0..n_local-1 and seeded random offsets, n_slash in all. Both lists are
+    shuffled (their order carries no meaning). Returns (v_idx [B,Hq,n_vertical],
+    v_cnt [B,Hq], s_off [B,Hq,n_slash], s_cnt [B,Hq]), int32."""
+    G = spec.Hq // spec.Hkv
+    v_idx = np.empty((spec.B, spec.Hq, n_vertical), np.int32)
+    s_off = np.empty((spec.B, spec.Hq, n_slash), np.int32)
+    for b in range(spec.B):
+        for h in range(spec.Hq):
+            rng = _rng(seed, "vsidx", b, h)
+            fixed = list(dict.fromkeys([int(x) for x in _vertical_positions(spec, seed, b, h // G)] +
+                                       [0, 1, 2, 3]))[:n_vertical]
+            rest = np.setdiff1d(np.arange(spec.N), fixed)
+            vc = np.concatenate([fixed, rng.choice(rest, size=n_vertical - len(fixed), replace=False)])
+            local = np.arange(min(n_local, n_slash))
+            so = np.concatenate([local, rng.choice(np.arange(len(local), spec.N), size=n_slash - len(local),
+                                                   replace=False)])
+            v_idx[b, h] = rng.permutation(vc)
+            s_off[b, h] = rng.permutation(so)
+    cnt_v = np.full((spec.B, spec.Hq), n_vertical, np.int32)
+    cnt_s = np.full((spec.B, spec.Hq), n_slash, np.int32)
+    return v_idx, cnt_v, s_off, cnt_s

@@ -7,6 +7,8 @@
  *   [Stem] "Stem: Rethinking Causal Information Flow in Sparse Attention",
  *          Resumo técnico, 2. Metodologia A (TPD), B (OAM), Implementação.
  *   [ART]  "Resumo Técnico: ART (Attention Run-time Termination)", 2. Metodologia 2.1-2.4.
+ *   [VSP]  "VSPrefill: Vertical-Slash Sparse Attention with Lightweight Indexing for
+ *          Long-Context Prefilling", 2. Metodologia A (vertical-slash pattern), B.3 (fused kernel).
  *
  * The problem as those pages frame it: block scores -> per-tile top-k list
  * kv_idx -> sparse attention that streams only the listed blocks ([UGS] steps
@@ -206,6 +208,30 @@ bsa_status bsa_select(const bsa_shape* shape, const bsa_select_params* params,
 bsa_status bsa_attend(const bsa_shape* shape, const void* q, const void* k, const void* v,
                       const int32_t* kv_idx, const int32_t* kv_cnt, int W, float softmax_scale,
                       void* out, float* lse, int32_t* dev_status, void* stream);
+
+/* ---- vertical-slash sparse attention ([VSP] Metodologia A, B.3) ------------------- */
+
+/* Query row i of head (b, h) attends to the union, each key once, of the vertical
+ * columns j <= i and the keys i - o of the slash offsets o <= i:
+ *   O_i = sum over those keys j of softmax(scale * q_i.k_j) v_j.
+ *   v_idx [B,Hq,Wv] int32, device: vertical key positions (any order), the first
+ *         v_cnt[b,h] used;  s_off [B,Hq,Ws] int32, device: slash offsets (any order),
+ *         the first s_cnt[b,h] used. Entries outside [0, N) are skipped and reported
+ *         as BSA_DEV_BAD_INDEX; counts outside [0, width] are reported and clamped.
+ *   out like Q (bf16); lse [B,Hq,N] fp32 or NULL (-inf, with output 0, for a row
+ *         with no key).  dev_status device int32, required.
+ * The two index lists are merged per query tile into the ascending list of the key
+ * blocks that hold a kept key, and the attention masks every (row, key) pair by the
+ * rule above ([VSP] B.3 merges the vertical and diagonal indices in the kernel).
+ * Shapes: bf16, d 128, block_k 64, tile_q 128; Wv, Ws >= 1 and min(N/64, Wv + 3*Ws)
+ * <= 1024 (else BSA_ERR_UNSUPPORTED). Workspace: bsa_attend_vs_workspace_bytes()
+ * bytes, 256-byte aligned (0 for an unsupported shape). */
+size_t bsa_attend_vs_workspace_bytes(const bsa_shape* shape, int Wv, int Ws);
+bsa_status bsa_attend_vs(const bsa_shape* shape, const void* q, const void* k, const void* v,
+                         const int32_t* v_idx, const int32_t* v_cnt, int Wv,
+                         const int32_t* s_off, const int32_t* s_cnt, int Ws, float softmax_scale,
+                         void* out, float* lse, int32_t* dev_status, void* workspace,
+                         size_t workspace_bytes, void* stream);
 
 /* ---- decode with run-time termination ([ART] 2.1-2.4) ----------------------------- */
 

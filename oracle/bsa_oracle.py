@@ -20,6 +20,10 @@ Sources (summary pages, cited by title and section):
   (tile-wise streaming exposes the partial output O^(t)), 2.2 (probe vector,
   d_scale and d_direction against tau and phi), 2.3 (patience p), 2.4
   (block 0 always evaluated).
+* [VSP] "VSPrefill: Vertical-Slash Sparse Attention with Lightweight
+  Indexing for Long-Context Prefilling" -- 2. Metodologia A (vertical
+  columns and slash diagonals), B.3 (a fused kernel attends over the merged
+  vertical and diagonal indices).
 
 Conventions: inputs are bf16 values widened exactly to fp64 (or fp32 values
 widened); arithmetic is fp64 unless a step says fp32. Layouts: Q [B,Hq,N,d],
@@ -397,6 +401,51 @@ def dense_causal_attention(Q, K, V, scale):
     logits[np.triu(np.ones((N, N), bool), 1)] = -np.inf
     p = np.exp(logits - logits.max(axis=1, keepdims=True))
     return (p / p.sum(axis=1, keepdims=True)) @ V
+
+
+def vs_keys(i: int, v_cols: Sequence[int], s_offs: Sequence[int]) -> np.ndarray:
+    """Key positions of query row i under a vertical-slash pattern ([VSP,
+    Metodologia A]: vertical columns are keys every later query attends to; a
+    slash offset o is the diagonal of keys j = i - o): the union, each key once,
+    of {j in v_cols : j <= i} and {i - o : o in s_offs, o <= i}, ascending."""
+    keys = {int(j) for j in v_cols if 0 <= int(j) <= i}
+    keys.update(i - int(o) for o in s_offs if 0 <= int(o) <= i)
+    return np.array(sorted(keys), dtype=np.int64)
+
+
+def attend_vs(Q, K, V, v_idx, v_cnt, s_off, s_cnt, scale, rows=None):
+    """Softmax attention of every query row over its vertical-slash key set
+    ([VSP, Metodologia B.3]: the sparse attention over the merged vertical and
+    diagonal indices). Q [B,Hq,N,d], K/V [B,Hkv,N,d]; v_idx [B,Hq,Wv] and s_off
+    [B,Hq,Ws] with counts v_cnt, s_cnt [B,Hq]: entries beyond the count, and
+    entries outside [0, N), are ignored. Returns (O [B,Hq,N,d], lse [B,Hq,N]) in
+    fp64; a row with an empty key set has output 0 and lse -inf. With ``rows``
+    (a list of (b, h, i)) only those rows are computed, the rest left NaN."""
+    B, Hq, N, d = Q.shape
+    G = Hq // K.shape[1]
+    O = np.full((B, Hq, N, d), np.nan)
+    lse = np.full((B, Hq, N), np.nan)
+    if rows is None:
+        rows = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(N)]
+    cache = {}
+    for b, h, i in rows:
+        if (b, h) not in cache:
+            vc = [int(j) for j in v_idx[b, h, :int(v_cnt[b, h])] if 0 <= int(j) < N]
+            so = [int(o) for o in s_off[b, h, :int(s_cnt[b, h])] if 0 <= int(o) < N]
+            cache[b, h] = (vc, so, widen(K[b, h // G]), widen(V[b, h // G]), widen(Q[b, h]))
+        vc, so, Kf, Vf, Qf = cache[b, h]
+        keys = vs_keys(i, vc, so)
+        if keys.size == 0:
+            O[b, h, i] = 0.0
+            lse[b, h, i] = -np.inf
+            continue
+        logits = scale * (Kf[keys] @ Qf[i])
+        mx = logits.max()
+        p = np.exp(logits - mx)
+        den = p.sum()
+        O[b, h, i] = (p @ Vf[keys]) / den
+        lse[b, h, i] = mx + math.log(den)
+    return O, lse
 
 
 # ---------------------------------------------------------------------------

@@ -189,3 +189,22 @@ def test_selftest_mode_validation():
     L = bb.lib()
     assert L.bsa_selftest_wait(3, 16, 16, None) == bb.BSA_ERR_INVALID_ARG
     assert L.bsa_selftest_wait(0, None, 16, None) == bb.BSA_ERR_INVALID_ARG
+
+
+def test_attend_vs_validation():
+    L = bb.lib()
+    s = _shape(N=131072)
+    assert bb.bsa_attend_vs_workspace_bytes(s, 64, 64) > 0
+    assert bb.bsa_attend_vs_workspace_bytes(s, 64, 400) == 0          # 64 + 3*400 > 1024 lists
+    assert bb.bsa_attend_vs_workspace_bytes(_shape(N=32768), 512, 512) > 0   # capped at n_kb = 512
+    assert bb.bsa_attend_vs_workspace_bytes(_shape(d=64), 64, 64) == 0
+    assert bb.bsa_attend_vs_workspace_bytes(_shape(tile_q=64), 64, 64) == 0
+    assert bb.bsa_attend_vs_workspace_bytes(s, 0, 64) == 0
+    big = 1 << 34
+    assert L.bsa_attend_vs(ctypes.byref(s), 16, 16, 16, None, 16, 64, 16, 16, 64, 0.1, 16, None, 16, 256,
+                           big, None) == bb.BSA_ERR_INVALID_ARG
+    assert L.bsa_attend_vs(ctypes.byref(s), 16, 16, 16, 16, 16, 64, 16, 16, 400, 0.1, 16, None, 16, 256,
+                           big, None) == bb.BSA_ERR_UNSUPPORTED
+    assert L.bsa_attend_vs(ctypes.byref(s), 16, 16, 16, 16, 16, 64, 16, 16, 64, 0.1, 16, None, 16, 256,
+                           100, None) == bb.BSA_ERR_INVALID_ARG
+    assert b"workspace" in L.bsa_last_error()

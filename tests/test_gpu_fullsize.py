@@ -116,3 +116,21 @@ def test_full_decode_art_64k():
                                      1 / math.sqrt(128), spec.tau, spec.phi, 1, dims)
         agree += int(u_ref == u)
     assert agree >= 6
+    # repeated launches: every one must end without a device error (an early stop must never
+    # leave a wait to run out) and give the same blocks and bit-identical outputs
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    acc = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for tau, phi, p in ((spec.tau, spec.phi, 1), (float("inf"), float("inf"), 1), (float("inf"), float("inf"), 3)):
+        first = None
+        for _ in range(30):
+            o2, u2, _, st2 = bb.decode(qd, kd, vd, block_kv=128, tau=tau, phi=phi, patience=p,
+                                       probe_dims=dims)
+            acc.bitwise_or_(st2)
+            if first is None:
+                first = (o2.clone(), u2.clone())
+            else:
+                assert torch.equal(u2, first[1]) and torch.equal(o2, first[0])
+        torch.cuda.synchronize()
+        assert int(acc.item()) == 0, (tau, phi, p)
+        if tau == float("inf"):
+            assert (first[1] == p + 1).all()

@@ -525,6 +525,61 @@ def test_additive_value_term_closed_forms():
     assert np.array_equal(s[0, :, 3, 6], m[0, :, 3, 6]) and np.array_equal(s[0, :, 3, 7], m[0, :, 3, 7])
 
 
+def _vs_case(seed=21, N=256, d=16):
+    rng = np.random.default_rng(seed)
+    Q = S.f32_to_bf16_bits(rng.standard_normal((1, 2, N, d)).astype(np.float32))
+    K = S.f32_to_bf16_bits(rng.standard_normal((1, 1, N, d)).astype(np.float32))
+    V = S.f32_to_bf16_bits(rng.standard_normal((1, 1, N, d)).astype(np.float32))
+    return Q, K, V
+
+
+def _vs_lists(v, s, Hq=2):
+    vi = np.array([v] * Hq, np.int32)[None]
+    so = np.array([s] * Hq, np.int32)[None]
+    return vi, np.full((1, Hq), vi.shape[-1], np.int32), so, np.full((1, Hq), so.shape[-1], np.int32)
+
+
+def test_vs_every_diagonal_or_every_column_is_dense_causal():
+    Q, K, V = _vs_case()
+    N = 256
+    dense = O.dense_causal_attention(Q[0, 1], K[0, 0], V[0, 0], 0.25)
+    for v, s in ([[], list(range(N))], [list(range(N)), []], [list(range(N)), list(range(N))]):
+        vi, vc, so, sc = _vs_lists(v if v else [0], s if s else [0])
+        if not v:
+            vc[:] = 0
+        if not s:
+            sc[:] = 0
+        o, lse = O.attend_vs(Q, K, V, vi, vc, so, sc, 0.25)
+        np.testing.assert_allclose(o[0, 1], dense, atol=1e-12)   # union: no key counted twice
+
+
+def test_vs_single_diagonal_returns_own_value():
+    """S = {0}, no vertical columns: each row attends only to itself, O_i = v_i."""
+    Q, K, V = _vs_case()
+    vi, vc, so, sc = _vs_lists([0], [0])
+    vc[:] = 0
+    o, lse = O.attend_vs(Q, K, V, vi, vc, so, sc, 0.25)
+    np.testing.assert_array_equal(o[0, 0], O.widen(V[0, 0]))
+    np.testing.assert_allclose(lse[0, 0], 0.25 * np.einsum("nd,nd->n", O.widen(Q[0, 0]), O.widen(K[0, 0])),
+                               atol=1e-12)
+
+
+def test_vs_key_sets_and_empty_rows():
+    assert list(O.vs_keys(10, [0, 3, 11, 40], [0, 2, 10, 20])) == [0, 3, 8, 10]
+    assert list(O.vs_keys(1, [5], [4])) == []
+    Q, K, V = _vs_case()
+    vi, vc, so, sc = _vs_lists([100], [64])
+    o, lse = O.attend_vs(Q, K, V, vi, vc, so, sc, 0.25)
+    assert not o[0, 0, :64].any() and np.isneginf(lse[0, 0, :64]).all()     # nothing visible yet
+    np.testing.assert_array_equal(o[0, 0, 64], O.widen(V[0, 0, 0]))      # only key 0 = 64 - 64
+    # rows 100..163: key 100 and key i - 64 (distinct) -> a two-key softmax
+    i = 120
+    ks = [56, 100]
+    lg = 0.25 * (O.widen(K[0, 0, ks]) @ O.widen(Q[0, 0, i]))
+    p = np.exp(lg - lg.max())
+    np.testing.assert_allclose(o[0, 0, i], (p @ O.widen(V[0, 0, ks])) / p.sum(), atol=1e-12)
+
+
 def test_decode_list_in_order_matches_decode():
     """Visiting blocks 0, 1, ... through the list form gives the in-order decode."""
     q, Kc, Vc = _decode_case()
