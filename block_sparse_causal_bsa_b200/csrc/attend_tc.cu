@@ -6,37 +6,33 @@
 // with an online softmax. Shapes: bf16, d = 128, key blocks of 64, query
 // tiles of 128.
 //
-// One CTA per (batch, query head, query tile); 352 threads in four roles:
-//   warp 0 (one thread)  TMA producer: the Q tile once, then K and V tiles of
-//                        128 keys = two listed blocks gathered into adjacent
-//                        shared-memory rows, two stages deep.
-//   warps 1, 10          MMA issuers, one thread each, one per half tile (= one
-//                        listed block): S_h = Q K_h^T (N = 64) into the half's
-//                        part of one of two TMEM S buffers (the next tile's S_h is
-//                        issued before this tile's value product), then
-//                        O_h += P_h V_h into the half's own TMEM accumulator once
-//                        the half's P is written, with P_h read straight from
-//                        tensor memory. The two halves run as separate pipelines.
-//   warps 2-9            softmax: two warps per TMEM lane quarter; a thread owns
-//                        half of one query row (the 64 keys of one listed block)
-//                        and runs an independent online softmax over the blocks
-//                        it sees: running max and sum of its half only, its own
-//                        O_h accumulator, rescaled in TMEM only when its running
-//                        max grew by more than 2^8 (exact: l and O keep the same
-//                        stale max). No per-tile exchange between the halves.
-//                        P_h (bf16, two per 32-bit column) is stored with
-//                        tcgen05.st over the first 32 columns of the half's S
-//                        region, which the softmax has just read.
-//                        Epilogue: the two halves meet once, through shared
-//                        memory: m = max(m0, m1), l = l0 2^(m0-m) + l1 2^(m1-m),
-//                        O = (O_0 2^(m0-m) + O_1 2^(m1-m)) / l  -- the exact merge
-//                        of two softmax partial sums; each half writes 64 of the
-//                        128 output columns (and lse).
+// One CTA per (batch, query head, query tile), 192 threads, two CTAs per SM
+// (256 TMEM columns and ~100 KB of shared memory each), so that every SM runs
+// two independent pipelines of different tiles: one CTA's prologue, epilogue
+// and softmax phases overlap the other's tensor-core work.
+//   warp 0 (one thread)  TMA producer: the Q tile once, then the K and V rows of
+//                        one listed block per stage, two stages deep.
+//   warp 1 (one thread)  MMA issuer: S_j = Q K_j^T (M128 N64, 8 x K16) into one
+//                        of two TMEM S buffers -- S_{j+1} is issued before the
+//                        value product of block j -- then O += P_j V_j once P_j
+//                        is written, P_j read straight from tensor memory (the
+//                        A operand) and V as an MN-major B operand.
+//   warps 2-5            softmax, one per TMEM lane quarter, a thread per query
+//                        row: 64 S values from TMEM, the causal mask on the
+//                        diagonal block, running max and sum, O rescaled in TMEM
+//                        only when the running max grew by more than 2^8 (exact:
+//                        l and O keep the same stale max), ex2 exponentials, P
+//                        (bf16, two per 32-bit column) stored with tcgen05.st over
+//                        the first 32 columns of the S buffer just read. O / l and
+//                        lse use the sum l of the fp32 exponentials; rows of the
+//                        vertical-slash variant (possibly a handful of keys) divide
+//                        O by the sum of the bf16 weights as applied instead.
+//                        Epilogue: O / l to bf16 in global memory, and the lse.
 // Shared-memory operand layouts (128-byte swizzled, as TMA writes them):
 //   Q, K: K-major [rows x 64 elements] halves; V: MN-major (rows = keys, 64
-//   contiguous head dims per 128-byte row).
-// TMEM: S buffers at columns 0 and 128 (half h at +64h; its P over the first 32
-// of those columns once read), O_0 at 256, O_1 at 384.
+//   contiguous head dims per 128-byte row), the two 64-dim halves 8 KB apart.
+// TMEM (256 columns): O at 0, S buffers at 128 and 192 (P over the first 32
+// columns of a buffer once read).
 // The CTA-to-work mapping walks (batch, KV head) outermost and the query heads
 // of a group innermost, so CTAs running together gather from one KV head and
 // reuse its blocks through L2.
@@ -61,35 +57,31 @@ constexpr int BQ = 128;          // query rows per tile
 constexpr int BKB = 64;          // keys per listed block
 constexpr int HD = 128;          // head dim
 constexpr int NS = 2;            // K/V pipeline stages
-constexpr int kThreads = 352;
-constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 4;
 constexpr int kMaxList = 1024;   // kv_idx entries staged per tile
-constexpr uint32_t kHalf = 16384;            // [128 rows x 128 bytes]
-constexpr uint32_t kTile = 2 * kHalf;        // 128 rows x 128 dims bf16
-constexpr uint32_t kBoxK = 8192;             // one 64-key block half
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;                // S buffers at columns 0 and 128
-constexpr uint32_t kColO = 256;              // O_0 at 256, O_1 at 384
+constexpr uint32_t kQHalf = 16384;           // Q: [128 rows x 128 bytes] per 64-dim half
+constexpr uint32_t kBHalf = 8192;            // K or V block: [64 rows x 128 bytes] per 64-dim half
+constexpr uint32_t kBlock = 2 * kBHalf;      // one K or V block (64 keys x 128 dims)
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColO = 0;                // O accumulator
+constexpr uint32_t kColS = 128;              // S buffers at 128 and 192
 
 struct __align__(8) Ctrl {
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
-  uint64_t s_full[2][2];                 // [half][buffer]
-  uint64_t p_full[2], o_ready[2];         // per half tile
-  uint64_t done[2];
-  uint64_t lbar[4];                 // per lane quarter: both halves' (m, l) written (once)
+  uint64_t s_full[2];
+  uint64_t p_full, o_ready, done;
   uint32_t tmem;
   int abort_flag;
   int n_list;
-  float mpart[2][128];              // [half][row] final running max of the half
-  float lpart[2][128];              // [half][row] final row-sum part of the half
   int list[kMaxList];
 };
 
 constexpr size_t kSmemQ = 0;
-constexpr size_t kSmemK = kSmemQ + kTile;
-constexpr size_t kSmemV = kSmemK + NS * kTile;
-constexpr size_t kSmemCtrl = kSmemV + NS * kTile;
+constexpr size_t kSmemK = kSmemQ + 2 * kQHalf;
+constexpr size_t kSmemV = kSmemK + NS * kBlock;
+constexpr size_t kSmemCtrl = kSmemV + NS * kBlock;
 constexpr size_t kSmemBytes = kSmemCtrl + sizeof(Ctrl) + 1024;   // + alignment slack
 
 __device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
@@ -98,6 +90,14 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// (a0, a1) += (b0, b1) as one packed fp32x2 add (sm_100), rounding as two fadds
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
 }
 
 // Keys j0+u (u < 64) of block blk that row i keeps under the vertical-slash rule:
@@ -124,7 +124,7 @@ __device__ __forceinline__ uint64_t vs_keep(const unsigned long long* __restrict
 }  // namespace
 
 template <bool VS>
-__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
+__global__ void __launch_bounds__(kThreads, 2) attend_tc_kernel(
     const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
     const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ kv_idx,
     const int32_t* __restrict__ kv_cnt, int W, float scale_log2, uint16_t* __restrict__ out,
@@ -156,17 +156,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     tc::mbar_init(&c.q_full, 1);
     for (int s = 0; s < NS; ++s) {
       tc::mbar_init(&c.k_full[s], 1);
-      tc::mbar_init(&c.k_empty[s], 2);      // both halves' S products read the K tile
+      tc::mbar_init(&c.k_empty[s], 1);
       tc::mbar_init(&c.v_full[s], 1);
-      tc::mbar_init(&c.v_empty[s], 2);      // both halves' value products read the V tile
+      tc::mbar_init(&c.v_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      for (int bfi = 0; bfi < 2; ++bfi) tc::mbar_init(&c.s_full[i][bfi], 1);
-      tc::mbar_init(&c.p_full[i], kSoftmaxWarps / 2);
-      tc::mbar_init(&c.o_ready[i], 1);
-      tc::mbar_init(&c.done[i], 1);
-    }
-    for (int q = 0; q < 4; ++q) tc::mbar_init(&c.lbar[q], 2);
+    tc::mbar_init(&c.s_full[0], 1);
+    tc::mbar_init(&c.s_full[1], 1);
+    tc::mbar_init(&c.p_full, kSoftmaxWarps);
+    tc::mbar_init(&c.o_ready, 1);
+    tc::mbar_init(&c.done, 1);
     c.abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -198,57 +196,50 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
   tc::tc_fence_after();
   const uint32_t tmem = c.tmem;
   const int nl = c.n_list;
-  const int ntiles = (nl + 1) / 2;
   volatile int* abort_flag = &c.abort_flag;
-  int k_issued = 0, v_issued = 0;     // tiles whose K / V loads the producer issued
+  int k_issued = 0, v_issued = 0;     // blocks whose K / V loads the producer issued
   bool mma_issued = false;
 
-  if (warp == 0 && lane == 0 && ntiles > 0) {
+  if (warp == 0 && lane == 0 && nl > 0) {
     // ---------------- TMA producer ----------------
     tc::prefetch_tmap(&tmq);
     tc::prefetch_tmap(&tmk);
     tc::prefetch_tmap(&tmv);
-    tc::mbar_arrive_expect_tx(&c.q_full, kTile);
+    tc::mbar_arrive_expect_tx(&c.q_full, 2 * kQHalf);
     tc::tma_load_2d(sm + kSmemQ, &tmq, 0, q_row0, &c.q_full);
-    tc::tma_load_2d(sm + kSmemQ + kHalf, &tmq, 64, q_row0, &c.q_full);
-    for (int j = 0; j < ntiles; ++j) {
+    tc::tma_load_2d(sm + kSmemQ + kQHalf, &tmq, 64, q_row0, &c.q_full);
+    for (int j = 0; j < nl; ++j) {
       const int s = j % NS;
-      const int ja = c.list[2 * j];
-      const int jb = (2 * j + 1 < nl) ? c.list[2 * j + 1] : ja;
-      const int ra = kv_row0 + ja * BKB, rb = kv_row0 + jb * BKB;
+      const int r = kv_row0 + c.list[j] * BKB;
       if (j >= NS && !tc::mbar_wait(&c.k_empty[s], ((j / NS) - 1) & 1, abort_flag, dev_status)) break;
-      uint8_t* kd = sm + kSmemK + s * kTile;
-      tc::mbar_arrive_expect_tx(&c.k_full[s], kTile);
-      tc::tma_load_2d(kd, &tmk, 0, ra, &c.k_full[s]);
-      tc::tma_load_2d(kd + kBoxK, &tmk, 0, rb, &c.k_full[s]);
-      tc::tma_load_2d(kd + kHalf, &tmk, 64, ra, &c.k_full[s]);
-      tc::tma_load_2d(kd + kHalf + kBoxK, &tmk, 64, rb, &c.k_full[s]);
+      uint8_t* kd = sm + kSmemK + s * kBlock;
+      tc::mbar_arrive_expect_tx(&c.k_full[s], kBlock);
+      tc::tma_load_2d(kd, &tmk, 0, r, &c.k_full[s]);
+      tc::tma_load_2d(kd + kBHalf, &tmk, 64, r, &c.k_full[s]);
       k_issued = j + 1;
       if (j >= NS && !tc::mbar_wait(&c.v_empty[s], ((j / NS) - 1) & 1, abort_flag, dev_status)) break;
-      uint8_t* vd = sm + kSmemV + s * kTile;
-      tc::mbar_arrive_expect_tx(&c.v_full[s], kTile);
-      tc::tma_load_2d(vd, &tmv, 0, ra, &c.v_full[s]);
-      tc::tma_load_2d(vd + kBoxK, &tmv, 0, rb, &c.v_full[s]);
-      tc::tma_load_2d(vd + kHalf, &tmv, 64, ra, &c.v_full[s]);
-      tc::tma_load_2d(vd + kHalf + kBoxK, &tmv, 64, rb, &c.v_full[s]);
+      uint8_t* vd = sm + kSmemV + s * kBlock;
+      tc::mbar_arrive_expect_tx(&c.v_full[s], kBlock);
+      tc::tma_load_2d(vd, &tmv, 0, r, &c.v_full[s]);
+      tc::tma_load_2d(vd + kBHalf, &tmv, 64, r, &c.v_full[s]);
       v_issued = j + 1;
     }
-  } else if ((warp == 1 || warp == 10) && lane == 0 && ntiles > 0) {
-    // ---------------- MMA issuer of one half ----------------
-    const int hf = warp == 1 ? 0 : 1;
+  } else if (warp == 1 && lane == 0 && nl > 0) {
+    // ---------------- MMA issuer ----------------
     constexpr uint32_t idS = tc::idesc_bf16_f32(128, 64, false, false);
     constexpr uint32_t idPV = tc::idesc_bf16_f32(128, 128, false, true);
     auto issue_s = [&](int j) {
-      // S_h = Q (128 x d) . K_h^T, K_h = rows 64*hf .. 64*hf+63 of the K tile
-      const uint32_t kb = sK + (j % NS) * kTile + hf * kBoxK;
-      const uint32_t d = tmem + kColS + (j % 2) * 128 + hf * 64;
+      // S_j = Q (128 x d) . K_j^T
+      const uint32_t kb = sK + (j % NS) * kBlock;
+      const uint32_t d = tmem + kColS + (j % 2) * 64;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-        tc::umma_bf16(d, tc::sdesc_sw128(sQ + off, 16, 1024), tc::sdesc_sw128(kb + off, 16, 1024), idS,
+        const uint32_t qoff = (kk >> 2) * kQHalf + (kk & 3) * 32;
+        const uint32_t koff = (kk >> 2) * kBHalf + (kk & 3) * 32;
+        tc::umma_bf16(d, tc::sdesc_sw128(sQ + qoff, 16, 1024), tc::sdesc_sw128(kb + koff, 16, 1024), idS,
                       kk > 0);
       }
-      tc::umma_commit(&c.s_full[hf][j % 2]);
+      tc::umma_commit(&c.s_full[j % 2]);
       tc::umma_commit(&c.k_empty[j % NS]);
     };
     bool ok = tc::mbar_wait(&c.q_full, 0, abort_flag, dev_status) &&
@@ -258,78 +249,73 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
       issue_s(0);
       mma_issued = true;
     }
-    for (int j = 0; ok && j < ntiles; ++j) {
+    for (int j = 0; ok && j < nl; ++j) {
       const int jn = j + 1;
-      if (jn < ntiles) {
-        // S_h(jn) overwrites the buffer of tile jn-2, whose P this half's value
-        // product of tile jn-2 = j-1 reads: wait for that product to complete
-        // (which also implies the softmax read S there)
+      if (jn < nl) {
+        // S(jn) overwrites the buffer of block jn-2, whose P the value product of block
+        // jn-2 = j-1 reads: wait for that product to complete (which also implies the
+        // softmax read S there)
         ok = tc::mbar_wait(&c.k_full[jn % NS], (jn / NS) & 1, abort_flag, dev_status) &&
-             (jn < 2 || tc::mbar_wait(&c.o_ready[hf], (jn - 2) & 1, abort_flag, dev_status));
+             (jn < 2 || tc::mbar_wait(&c.o_ready, (jn - 2) & 1, abort_flag, dev_status));
         if (!ok) break;
         tc::tc_fence_after();
         issue_s(jn);
       }
       ok = tc::mbar_wait(&c.v_full[j % NS], (j / NS) & 1, abort_flag, dev_status) &&
-           tc::mbar_wait(&c.p_full[hf], j & 1, abort_flag, dev_status);
+           tc::mbar_wait(&c.p_full, j & 1, abort_flag, dev_status);
       if (!ok) break;
       tc::tc_fence_after();
-      const uint32_t vb = sV + (j % NS) * kTile;
-      const uint32_t pa = tmem + kColS + (j % 2) * 128 + hf * 64;    // P_h in TMEM
-      // O_h += P_h (128 rows x 64 keys) . V rows of this half's block
+      const uint32_t vb = sV + (j % NS) * kBlock;
+      const uint32_t pa = tmem + kColS + (j % 2) * 64;              // P_j in TMEM
+      // O += P_j (128 rows x 64 keys) . V_j (64 keys x 128 dims)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        tc::umma_bf16_ts(tmem + kColO + hf * 128, pa + kk * 8,
-                         tc::sdesc_sw128(vb + (hf * 4 + kk) * 2048, kHalf, 1024), idPV,
+        tc::umma_bf16_ts(tmem + kColO, pa + kk * 8, tc::sdesc_sw128(vb + kk * 2048, kBHalf, 1024), idPV,
                          (j > 0 || kk > 0) ? 1u : 0u);
       }
-      tc::umma_commit(&c.o_ready[hf]);
+      tc::umma_commit(&c.o_ready);
       tc::umma_commit(&c.v_empty[j % NS]);
     }
-  } else if (warp >= 2 && warp <= 9) {
+  } else if (warp >= 2) {
     // ---------------- softmax warps ----------------
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;                   // 0: keys 0-63 of the tile, 1: keys 64-127
     const int r = quarter * 32 + lane;                  // row in the tile == TMEM lane
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t colO = kColO + half * 128;
     const int row_abs = t * BQ + r;
     const unsigned long long* vrow = VS ? vbits + bh * (size_t)(N / 64 + 1) : nullptr;
     const unsigned long long* srow = VS ? sbits + bh * (size_t)(N / 64 + 1) : nullptr;
-    float m_used = -INFINITY;                           // running max of this half, scaled log2 units
-    float l = 0.f;                                      // running sum of this half
+    float m_used = -INFINITY;                           // running max, scaled log2 units
+    float l = 0.f;                                      // running sum of the exponentials (lse)
+    float lq = 0.f;                                     // ... of their bf16 values (normalises O)
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      ok = warp_all(tc::mbar_wait(&c.s_full[half][j % 2], (j / 2) & 1, abort_flag, dev_status));
+    for (int j = 0; j < nl; ++j) {
+      ok = warp_all(tc::mbar_wait(&c.s_full[j % 2], (j / 2) & 1, abort_flag, dev_status));
       if (!ok) break;
       tc::tc_fence_after();
       float s[64];
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32];
-        tc::tmem_ld32(tl + kColS + (j % 2) * 128 + half * 64 + cc * 32, v);
+        tc::tmem_ld32(tl + kColS + (j % 2) * 64 + cc * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(v[i]);
       }
-      const bool has_b = 2 * j + 1 < nl;
-      const int blk = half == 0 ? c.list[2 * j] : (has_b ? c.list[2 * j + 1] : -1);
-      // mask: keys after this row, and the empty second slot of an odd tail
-      const bool diag = blk < 0 || blk * BKB + BKB - 1 > t * BQ;
+      const int blk = c.list[j];
       float mx8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
       if (VS) {
-        const uint64_t keep = blk < 0 ? 0ull : vs_keep(vrow, srow, row_abs, blk);
+        const uint64_t keep = vs_keep(vrow, srow, row_abs, blk);
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           s[i] = ((keep >> i) & 1ull) ? s[i] : -INFINITY;
           mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
         }
-      } else if (diag) {
+      } else if (blk * BKB + BKB - 1 > t * BQ) {
+        // the block reaches past the tile's first row: mask keys after this row
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          const bool vis = blk >= 0 && blk * BKB + i <= row_abs;
-          s[i] = vis ? s[i] : -INFINITY;
+          s[i] = blk * BKB + i <= row_abs ? s[i] : -INFINITY;
           mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
         }
       } else {
@@ -346,6 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
       }
       const float m_safe = (m_used == -INFINITY) ? 0.f : m_used;
       float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
+      float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 64; i += 4) {
@@ -353,89 +340,86 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const float p1 = ex2(fmaf(s[i + 1], scale_log2, -m_safe));
         const float p2 = ex2(fmaf(s[i + 2], scale_log2, -m_safe));
         const float p3 = ex2(fmaf(s[i + 3], scale_log2, -m_safe));
-        sum0 += p0; sum1 += p1; sum2 += p2; sum3 += p3;
         __nv_bfloat162 a = __floats2bfloat162_rn(p0, p1);
         __nv_bfloat162 bq = __floats2bfloat162_rn(p2, p3);
-        pk[i / 2] = *reinterpret_cast<uint32_t*>(&a);
-        pk[i / 2 + 1] = *reinterpret_cast<uint32_t*>(&bq);
+        const uint32_t wa = *reinterpret_cast<uint32_t*>(&a), wb = *reinterpret_cast<uint32_t*>(&bq);
+        pk[i / 2] = wa;
+        pk[i / 2 + 1] = wb;
+        add2(sum0, sum1, p0, p1);
+        add2(sum2, sum3, p2, p3);
+        if (VS) {
+          // vertical-slash rows may see a handful of keys: O is normalised by the sum of
+          // the bf16 weights the value product uses, so the applied weights sum to one (a
+          // row with one key gets exactly its value); block rows see >= 64 keys and use l
+          add2(q0, q1, __uint_as_float(wa << 16), __uint_as_float(wa & 0xffff0000u));
+          add2(q2, q3, __uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u));
+        }
       }
       l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
+      if (VS) lq = lq * alpha + ((q0 + q1) + (q2 + q3));
 
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // rescaling O_h: the previous value product of this half must have landed
-        ok = warp_all(tc::mbar_wait(&c.o_ready[half], (j - 1) & 1, abort_flag, dev_status));
+      if (j > 0) {
+        // the previous value product has landed: O may be rescaled, and the issuer has
+        // consumed p_full(j-1), so this warp's arrival below is for phase j (a parity wait
+        // cannot tell phase j-1 from j+1)
+        ok = warp_all(tc::mbar_wait(&c.o_ready, (j - 1) & 1, abort_flag, dev_status));
         if (!ok) break;
         tc::tc_fence_after();
+      }
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t v[32];
-          tc::tmem_ld32(tl + colO + cc * 32, v);
+          tc::tmem_ld32(tl + kColO + cc * 32, v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-          tc::tmem_st32(tl + colO + cc * 32, v);
+          tc::tmem_st32(tl + kColO + cc * 32, v);
         }
       }
-      // P_h -> TMEM over the first 32 columns of this half's (already read) S region
-      tc::tmem_st32(tl + kColS + (j % 2) * 128 + half * 64, pk);
+      // P -> TMEM over the first 32 columns of the (already read) S buffer
+      tc::tmem_st32(tl + kColS + (j % 2) * 64, pk);
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&c.p_full[half]);
+      if (lane == 0) tc::mbar_arrive(&c.p_full);
     }
-    // epilogue: merge the two halves' partial softmax sums, store 64 columns each
-    uint16_t* orow = out + ((size_t)bh * N + (size_t)t * BQ + r) * HD + half * 64;
-    bool have = ok && ntiles > 0;
-    if (have) have = warp_all(tc::mbar_wait(&c.o_ready[half], (ntiles - 1) & 1, abort_flag, dev_status));
-    if (ntiles > 0) {
-      c.mpart[half][r] = m_used;
-      c.lpart[half][r] = l;
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&c.lbar[quarter]);
-      // each half arrives only after its own last value product completed, so past
-      // this barrier both O accumulators are final
-      if (have) have = warp_all(tc::mbar_wait(&c.lbar[quarter], 0, abort_flag, dev_status));
-    }
+    // epilogue
+    uint16_t* orow = out + ((size_t)bh * N + (size_t)t * BQ + r) * HD;
+    bool have = ok && nl > 0;
+    if (have) have = warp_all(tc::mbar_wait(&c.o_ready, (nl - 1) & 1, abort_flag, dev_status));
     if (have) {
       tc::tc_fence_after();
-      const float m0 = c.mpart[0][r], m1 = c.mpart[1][r];
-      const float mm = fmaxf(m0, m1);
-      const float f0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - mm);
-      const float f1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - mm);
-      const float lt = c.lpart[0][r] * f0 + c.lpart[1][r] * f1;
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      const float w0 = f0 * inv, w1 = f1 * inv;
+      const float ln = VS ? lq : l;
+      const float inv = ln > 0.f ? 1.f / ln : 0.f;
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v0[32], v1[32];
-        tc::tmem_ld32(tl + kColO + half * 64 + cc * 32, v0);          // O_0, this half's columns
-        tc::tmem_ld32(tl + kColO + 128 + half * 64 + cc * 32, v1);    // O_1, same columns
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tc::tmem_ld32(tl + kColO + cc * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int k0 = i + 2 * e;
-            __nv_bfloat162 p = __floats2bfloat162_rn(
-                __uint_as_float(v0[k0]) * w0 + __uint_as_float(v1[k0]) * w1,
-                __uint_as_float(v0[k0 + 1]) * w0 + __uint_as_float(v1[k0 + 1]) * w1);
+            __nv_bfloat162 p = __floats2bfloat162_rn(__uint_as_float(v[i + 2 * e]) * inv,
+                                                     __uint_as_float(v[i + 2 * e + 1]) * inv);
             w[e] = *reinterpret_cast<uint32_t*>(&p);
           }
           *reinterpret_cast<uint4*>(orow + cc * 32 + i) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      if (lse && half == 0)
-        lse[bh * N + (size_t)t * BQ + r] = lt > 0.f ? (mm + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-    } else if (ntiles == 0) {
+      if (lse)
+        lse[bh * N + (size_t)t * BQ + r] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    } else if (nl == 0) {
 #pragma unroll
-      for (int i = 0; i < 64; i += 8)
+      for (int i = 0; i < HD; i += 8)
         *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
-      if (lse && half == 0) lse[bh * N + (size_t)t * BQ + r] = -INFINITY;
+      if (lse) lse[bh * N + (size_t)t * BQ + r] = -INFINITY;
     }
   }
 
   // ---------------- teardown ----------------
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 0 && lane == 0 && ntiles > 0) {
+  if (warp == 0 && lane == 0 && nl > 0) {
     // make sure no TMA copy of this CTA is still landing in shared memory: wait for
     // the last phase issued on every stage (earlier phases completed before it)
     tc::mbar_wait_timed(&c.q_full, 0);
@@ -444,14 +428,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     for (int j = v_issued - NS < 0 ? 0 : v_issued - NS; j < v_issued; ++j)
       tc::mbar_wait_timed(&c.v_full[j % NS], (j / NS) & 1);
   }
-  if ((warp == 1 || warp == 10) && lane == 0 && mma_issued) {
-    // every MMA this thread issued has completed once this commit arrives
-    const int hf = warp == 1 ? 0 : 1;
-    tc::umma_commit(&c.done[hf]);
-    tc::mbar_wait_timed(&c.done[hf], 0);
-  }
-  __syncthreads();
   if (warp == 1) {
+    if (lane == 0 && mma_issued) {
+      // every MMA this thread issued has completed once this commit arrives
+      tc::umma_commit(&c.done);
+      tc::mbar_wait_timed(&c.done, 0);
+    }
+    __syncwarp();
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
