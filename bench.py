@@ -332,8 +332,18 @@ def main_gpu(args):
     assert int(st_sel.item()) == 0 and int(st_att.item()) == 0 and int(st_score.item()) == 0
     sel_blocks = int(kv_cnt.sum().item())
     flops = 4.0 * spec.tile_q * spec.block_k * d * sel_blocks
-    # unmasked (i, j) pairs of the selected blocks, for the alternative count
-    triggered = None
+    # unmasked (i, j) pairs of the selected blocks (j <= i), for the alternative count: a block
+    # wholly below the tile's first row contributes tile_q * block_k pairs, a diagonal block fewer
+    kvl = kv_idx.long()
+    valid = torch.arange(W, device=dev)[None, None, None, :] < kv_cnt[..., None]
+    first_row = (torch.arange(n_qt, device=dev) * spec.tile_q)[None, None, :, None]
+    # pairs (r, c) with key j0 + c <= row i0 + r, r < tile_q, c < block_k
+    pairs = torch.zeros_like(kvl, dtype=torch.float64)
+    for r in range(spec.tile_q):
+        lim = (first_row + r - kvl * spec.block_k)                   # keys c <= lim are visible
+        pairs += (lim + 1).clamp(0, spec.block_k).double()
+    unmasked_pairs = float((pairs * valid).sum().item())
+    del kvl, valid, first_row, pairs
     launches_per_step = 6     # pool, score, select_rank, gate, finalize, attend
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -513,7 +523,9 @@ def main_gpu(args):
                                                                 world, dev)
     if rank == 0:
         sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         achieved = flops / (attend_ms * 1e-3) / 1e12
+        achieved_unmasked = 4.0 * d * unmasked_pairs / (attend_ms * 1e-3) / 1e12
         traffic = None
         tp = os.path.join(ROOT, "profiles", "attend_traffic.json")
         if os.path.exists(tp):
@@ -538,6 +550,12 @@ def main_gpu(args):
             "kernel_ms": {"score": score_ms, "select": select_ms, "attend": attend_ms},
             "score_backbones_ms": score_kinds,
             "vertical_slash": vs_res,
+            "attend_detail": {"frac_of_burst_peak": achieved / burst, "burst_peak": burst,
+                              "frac_of_datasheet_dense": achieved / 2250.0,
+                              "unmasked_pair_tflops": achieved_unmasked,
+                              "unmasked_pairs": unmasked_pairs,
+                              "step_ms_median": float(np.median(per.sum(axis=1))),
+                              "attend_ms_median": float(np.median(per[:, 2]))},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained,
                          "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
                          "kernel": "attend",

@@ -83,17 +83,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Warp-wide wait: lane 0 polls, the warp takes its verdict. Lane 0's acquire is
-// passed on to the other lanes by the warp-synchronous shuffle.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* dev_status) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, dev_status) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
-}
-
 // Wait for a phase that an early stop may leave incomplete forever. Returns 0 when the
 // phase completed, 1 when *halt was raised first, 2 when the CTA aborts (abort flag) or
 // kTimeoutNs elapse (then BSA_DEV_TIMEOUT is set and the abort flag raised).
