@@ -334,16 +334,17 @@ def main_gpu(args):
     flops = 4.0 * spec.tile_q * spec.block_k * d * sel_blocks
     # unmasked (i, j) pairs of the selected blocks (j <= i), for the alternative count: a block
     # wholly below the tile's first row contributes tile_q * block_k pairs, a diagonal block fewer
+    # pairs (r, c) with key j0 + c <= row i0 + r: sum over r < tile_q of clamp(a + r, 0, bk),
+    # a = i0 - j0 + 1, in closed form (a run of x = 1..bk-1 plus bk for every x >= bk)
     kvl = kv_idx.long()
     valid = torch.arange(W, device=dev)[None, None, None, :] < kv_cnt[..., None]
-    first_row = (torch.arange(n_qt, device=dev) * spec.tile_q)[None, None, :, None]
-    # pairs (r, c) with key j0 + c <= row i0 + r, r < tile_q, c < block_k
-    pairs = torch.zeros_like(kvl, dtype=torch.float64)
-    for r in range(spec.tile_q):
-        lim = (first_row + r - kvl * spec.block_k)                   # keys c <= lim are visible
-        pairs += (lim + 1).clamp(0, spec.block_k).double()
-    unmasked_pairs = float((pairs * valid).sum().item())
-    del kvl, valid, first_row, pairs
+    a = (torch.arange(n_qt, device=dev) * spec.tile_q)[None, None, :, None] - kvl * spec.block_k + 1
+    bk, tq = spec.block_k, spec.tile_q
+    lo, hi = a.clamp(min=1), (a + tq - 1).clamp(max=bk - 1)
+    ramp = torch.where(lo <= hi, (lo + hi) * (hi - lo + 1) // 2, torch.zeros_like(a))
+    flat = bk * (a + tq - torch.maximum(a, torch.full_like(a, bk))).clamp(min=0)
+    unmasked_pairs = float(((ramp + flat) * valid).sum().item())
+    del kvl, valid, a, lo, hi, ramp, flat
     launches_per_step = 6     # pool, score, select_rank, gate, finalize, attend
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
