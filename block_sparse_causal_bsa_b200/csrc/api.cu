@@ -357,6 +357,8 @@ static bsa_status check_decode(const bsa_decode_shape* s, const bsa_decode_param
   if (s->d != 64 && s->d != 128) return fail(BSA_ERR_UNSUPPORTED, "d must be 64 or 128");
   if (s->block_kv != 64 && s->block_kv != 128) return fail(BSA_ERR_UNSUPPORTED, "block_kv must be 64 or 128");
   if (s->L % s->block_kv) return fail(BSA_ERR_INVALID_ARG, "L must be a multiple of block_kv");
+  if ((long long)s->B * s->Hkv * s->L >= (1ll << 31))
+    return fail(BSA_ERR_UNSUPPORTED, "B * Hkv * L must be below 2^31 (cache rows are int32 coordinates)");
   if (s->dtype != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "decode takes bf16 only");
   if (p->patience < 1) return fail(BSA_ERR_INVALID_ARG, "patience must be >= 1");
   if (p->n_probe < 1 || p->n_probe > bsa::kMaxProbe || !p->probe_dims)

@@ -122,7 +122,8 @@ typedef struct {
 } bsa_select_params;
 
 /* Decode problem: one query token per sequence, KV cache of length L.
- * d in {64,128}; block_kv in {64,128}; L a multiple of block_kv; Hq/Hkv <= 8. */
+ * d in {64,128}; block_kv in {64,128}; L a multiple of block_kv; Hq/Hkv in {1,2,4,8};
+ * B*Hkv*L < 2^31. */
 typedef struct {
   int B, Hq, Hkv, L, d, block_kv;
   bsa_dtype dtype;           /* BSA_BF16 only */

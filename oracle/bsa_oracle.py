@@ -41,11 +41,20 @@ first query head of the KV group; d_scale is the absolute difference of the
 probe norms; d_direction is 1 - cosine, taken as 1 when a norm is zero;
 termination is decided per (batch, KV head).
 
+Readings for the added paths: the additive Output-Aware Metric is taken at
+block level (the block's mean value vector for V_j, natural log, weight beta,
+no 1/sqrt(d) on the score); the K-min/K-max score is the tile max of
+sum_c max(q_c kmin_c, q_c kmax_c); a vertical-slash row attends to the union,
+each key once, of its vertical columns j <= i and the keys i - o of its slash
+offsets; a decode over a block list visits the list in order and never tests
+its first entry.
+
 Parity status: every function below is pinned by CPU tests against closed
 forms, library routines (torch scaled_dot_product_attention, numpy.quantile)
-or brute force -- except the exact termination block on random decode data,
-which the pages do not fix ("parity unpinned" for that value; the decision
-rule itself is pinned by hand-worked traces).
+or brute force (the K-min/K-max score against the maximum over all 2^d box
+corners) -- except the exact termination block on random decode data, which
+the pages do not fix ("parity unpinned" for that value; the decision rule
+itself is pinned by hand-worked traces).
 """
 from __future__ import annotations
 

@@ -208,3 +208,13 @@ def test_attend_vs_validation():
     assert L.bsa_attend_vs(ctypes.byref(s), 16, 16, 16, 16, 16, 64, 16, 16, 64, 0.1, 16, None, 16, 256,
                            100, None) == bb.BSA_ERR_INVALID_ARG
     assert b"workspace" in L.bsa_last_error()
+
+
+def test_decode_cache_too_large_rejected():
+    L = bb.lib()
+    ds = bb.DecodeShape(64, 32, 8, 1 << 22, 128, 128, bb.BSA_BF16)     # 2^31 cache rows
+    dims = (ctypes.c_int * 2)(0, 1)
+    dp = bb.DecodeParams(1e-3, 1e-4, 1, 1, 2, dims)
+    assert L.bsa_decode(ctypes.byref(ds), ctypes.byref(dp), 16, 16, 16, 0.1, 16, 16, None, 16,
+                        None) == bb.BSA_ERR_UNSUPPORTED
+    assert b"2^31" in L.bsa_last_error()
