@@ -1,7 +1,9 @@
 // Decode attention with run-time termination on Blackwell tensor cores
 // ([ART] 2.1-2.4): the KV cache of one (batch, KV head) is streamed block by
-// block, in order; after each block the normalised partial output O^(t) is
-// probed, and from block 1 on the stability test decides whether to stop.
+// block, in order (or in the order of a caller's visit list, compacted into
+// shared memory by warp 6 before the pipeline starts); after each block the
+// normalised partial output O^(t) is probed, and from the second visit step on
+// the stability test decides whether to stop.
 //
 // One CTA per (batch, KV head), 224 threads:
 //   warp 0 (one thread)  TMA producer: K and V blocks of 128 keys, a ring of
@@ -26,9 +28,12 @@
 // and the softmax warps produce P_{t+1} (two P buffers) before they fold D_t, so
 // the softmax of one block overlaps the value product of the previous one. The
 // decider judges block t while the softmax warps go on; they look at that
-// verdict only before folding D_{t+1}, and on a stop return the unfolded O^(t). After a stop the producer
-// and MMA threads are released through a halt flag; the CTA then waits for its
-// own copies and MMAs and frees TMEM. All waits are bounded.
+// verdict only before folding D_{t+1}, and on a stop return the unfolded O^(t).
+// After a stop the producer and MMA threads are released through a halt flag;
+// the MMA issuer may then never issue S_{t+2}, so the softmax warps' wait for it
+// also watches the halt flag, and the four warps act on one verdict (posted per
+// warp and joined through the bounded `vote` mbarrier). The CTA then waits for
+// its own copies and MMAs and frees TMEM. All waits are bounded.
 // Shapes: bf16, d = 128, KV blocks of 128, Hq/Hkv <= 8.
 #include <math.h>
 
