@@ -334,17 +334,7 @@ def main_gpu(args):
     flops = 4.0 * spec.tile_q * spec.block_k * d * sel_blocks
     # unmasked (i, j) pairs of the selected blocks (j <= i), for the alternative count: a block
     # wholly below the tile's first row contributes tile_q * block_k pairs, a diagonal block fewer
-    # pairs (r, c) with key j0 + c <= row i0 + r: sum over r < tile_q of clamp(a + r, 0, bk),
-    # a = i0 - j0 + 1, in closed form (a run of x = 1..bk-1 plus bk for every x >= bk)
-    kvl = kv_idx.long()
-    valid = torch.arange(W, device=dev)[None, None, None, :] < kv_cnt[..., None]
-    a = (torch.arange(n_qt, device=dev) * spec.tile_q)[None, None, :, None] - kvl * spec.block_k + 1
-    bk, tq = spec.block_k, spec.tile_q
-    lo, hi = a.clamp(min=1), (a + tq - 1).clamp(max=bk - 1)
-    ramp = torch.where(lo <= hi, (lo + hi) * (hi - lo + 1) // 2, torch.zeros_like(a))
-    flat = bk * (a + tq - torch.maximum(a, torch.full_like(a, bk))).clamp(min=0)
-    unmasked_pairs = float(((ramp + flat) * valid).sum().item())
-    del kvl, valid, a, lo, hi, ramp, flat
+    unmasked_pairs = unmasked_pair_count(torch, kv_idx, kv_cnt, spec.tile_q, spec.block_k)
     launches_per_step = 6     # pool, score, select_rank, gate, finalize, attend
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -574,6 +564,21 @@ def main_gpu(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def unmasked_pair_count(torch, kv_idx, kv_cnt, tile_q, block_k):
+    """Number of (query row, key) pairs with key <= row inside the listed blocks: a block
+    starting at key j0 in the tile whose first row is i0 contributes, over rows r < tile_q,
+    clamp(a + r, 0, block_k) with a = i0 - j0 + 1 -- in closed form a ramp 1..block_k-1
+    plus block_k for every row past it. kv_idx [B,Hq,n_qt,W] and kv_cnt [B,Hq,n_qt]."""
+    W, n_qt = kv_idx.shape[-1], kv_idx.shape[-2]
+    kvl = kv_idx.long()
+    valid = torch.arange(W, device=kv_idx.device)[None, None, None, :] < kv_cnt[..., None]
+    a = (torch.arange(n_qt, device=kv_idx.device) * tile_q)[None, None, :, None] - kvl * block_k + 1
+    lo, hi = a.clamp(min=1), (a + tile_q - 1).clamp(max=block_k - 1)
+    ramp = torch.where(lo <= hi, (lo + hi) * (hi - lo + 1) // 2, torch.zeros_like(a))
+    flat = block_k * (a + tile_q - torch.maximum(a, torch.full_like(a, block_k))).clamp(min=0)
+    return float(((ramp + flat) * valid).sum().item())
 
 
 def _attend_sha():

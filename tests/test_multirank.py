@@ -1,8 +1,10 @@
-"""The N>1 path on CPU: two gloo ranks run the benchmark's rank-level logic
-(independent problems per rank, max-over-ranks timing, summed work)."""
+"""The benchmark's host logic on CPU: two gloo ranks run its rank-level logic
+(independent problems per rank, max-over-ranks timing, summed work), and its
+count of unmasked (row, key) pairs is checked against enumeration."""
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -49,3 +51,27 @@ def test_two_ranks_reduce_and_seed():
     for rank, (step, att, e2e, fl), seed in res:
         assert step == 11.0 and att == 10.0 and e2e == 20.0 and fl == 3e12
     assert res[0][2] != res[1][2]      # independent problems per rank
+
+
+def test_unmasked_pair_count_matches_brute_force():
+    """The bench's count of unmasked (row, key) pairs, against enumeration on small lists."""
+    import itertools
+    import bench as B
+    rng = np.random.default_rng(9)
+    for tq, bk in ((128, 64), (64, 64), (128, 128), (64, 128)):
+        n_qt, W = 6, 5
+        kv = np.full((1, 2, n_qt, W), -1, np.int32)
+        cnt = np.zeros((1, 2, n_qt), np.int32)
+        for h, t in itertools.product(range(2), range(n_qt)):
+            J = ((t + 1) * tq - 1) // bk
+            c = int(rng.integers(0, min(W, J + 1) + 1))
+            kv[0, h, t, :c] = rng.permutation(J + 1)[:c]
+            cnt[0, h, t] = c
+        got = B.unmasked_pair_count(torch, torch.from_numpy(kv), torch.from_numpy(cnt), tq, bk)
+        ref = 0
+        for h, t in itertools.product(range(2), range(n_qt)):
+            for w in range(cnt[0, h, t]):
+                j0 = int(kv[0, h, t, w]) * bk
+                rows = t * tq + np.arange(tq)[:, None]
+                ref += int((j0 + np.arange(bk)[None, :] <= rows).sum())
+        assert got == ref, (tq, bk, got, ref)

@@ -659,6 +659,21 @@ def test_decode_block_list_generator():
         assert len(set(row)) == 9 and (np.diff(row[1:]) < 0).all() and row[1:].min() >= 1
 
 
+def test_vs_index_generator():
+    """Synthetic vertical-slash indices: distinct, in range, the KV head's planted anchors and the
+    first four positions among the vertical columns, the local band among the slash offsets."""
+    spec = S.WORKLOADS["prefill_32k_vs"].scaled(N=4096, Hq=4, Hkv=2)
+    v, vc, so, sc = S.vs_indices(spec, 11, n_vertical=24, n_slash=20, n_local=8)
+    assert v.shape == (1, 4, 24) and so.shape == (1, 4, 20)
+    assert (vc == 24).all() and (sc == 20).all()
+    for h in range(4):
+        assert len(set(v[0, h])) == 24 and len(set(so[0, h])) == 20
+        assert v[0, h].min() >= 0 and v[0, h].max() < 4096 and so[0, h].min() >= 0 and so[0, h].max() < 4096
+        anchors = set(int(x) for x in S._vertical_positions(spec, 11, 0, h // 2))
+        assert anchors | {0, 1, 2, 3} <= set(int(x) for x in v[0, h])
+        assert set(range(8)) <= set(int(x) for x in so[0, h])
+
+
 def test_generator_structure():
     """The seeded generators plant the stated structure (not method arithmetic)."""
     spec = S.WORKLOADS["gated_prefill_128k"].scaled(N=4096, Hq=4, Hkv=1)
