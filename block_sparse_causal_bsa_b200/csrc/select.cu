@@ -494,8 +494,17 @@ __global__ void __launch_bounds__(1024) gate_kernel(const float* __restrict__ si
   const int total = B * n_qt;
   for (int i = threadIdx.x; i < total; i += blockDim.x) {
     const int b = i / n_qt, t = i % n_qt;
+    // eight heads' values in flight at a time, added in head order
     float acc = 0.0f;
-    for (int h = 0; h < Hq; ++h) acc = __fadd_rn(acc, sigma[((size_t)b * Hq + h) * n_qt + t]);
+    const float* col = sigma + (size_t)b * Hq * n_qt + t;
+    for (int h0 = 0; h0 < Hq; h0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = h0 + u < Hq ? __ldg(col + (size_t)(h0 + u) * n_qt) : 0.0f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (h0 + u < Hq) acc = __fadd_rn(acc, v[u]);
+    }
     const float sb = __fdiv_rn(acc, (float)Hq);
     sigma_bar[i] = sb;
     if (tile_slots(t, n_qt, tile_q, block_k, k_first, k_last, rho).cut) pop[atomicAdd(&cnt, 1u)] = sb;
