@@ -359,6 +359,15 @@ def main_gpu(args):
     step_ms = float(per.sum(axis=1).mean())
     score_ms, select_ms, attend_ms = (float(x) for x in per.mean(axis=0))
 
+    # warm variant: the same steps without the L2 flush in between
+    wevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(5)]
+    for i in range(5):
+        step(q, k, v, out, wevs[i])
+    torch.cuda.synchronize()
+    wper = np.array([[wevs[i][j].elapsed_time(wevs[i][j + 1]) for j in range(3)] for i in range(5)])
+    warm = {"step_ms": float(wper.sum(axis=1).mean()), "score_ms": float(wper[:, 0].mean()),
+            "select_ms": float(wper[:, 1].mean()), "attend_ms": float(wper[:, 2].mean())}
+
     # end to end through the C ABI with host buffers: every step copies its Q, K, V from
     # pinned host memory to the device and its O back, all inside the timed region. The
     # copies run on two copy streams with two device slots, so step i+1's host-to-device
@@ -575,7 +584,8 @@ def main_gpu(args):
                               "unmasked_pair_tflops": achieved_unmasked,
                               "unmasked_pairs": unmasked_pairs,
                               "step_ms_median": float(np.median(per.sum(axis=1))),
-                              "attend_ms_median": float(np.median(per[:, 2]))},
+                              "attend_ms_median": float(np.median(per[:, 2])),
+                              "warm_no_flush": warm},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained,
                          "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
                          "kernel": "attend",
