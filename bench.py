@@ -577,6 +577,7 @@ def main_gpu(args):
                        "l2": "256 MB buffer written between timed steps; inputs 1.6 GB > 126 MB L2",
                        "parallelism": f"independent problem per rank x{world}"},
             "kernel_ms": {"score": score_ms, "select": select_ms, "attend": attend_ms},
+            "path_rooflines": path_rooflines(spec, score_ms, select_ms, peaks),
             "score_backbones_ms": score_kinds,
             "vertical_slash": vs_res,
             "attend_detail": {"frac_of_burst_peak": achieved / burst, "burst_peak": burst,
@@ -590,8 +591,7 @@ def main_gpu(args):
                          "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
                          "kernel": "attend",
                          "peak_note": f"{peak_kind} sustained dense bf16 (kernel timed inside a step)"},
-            "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12 if world == 1 else
-                    total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "note": "pinned host buffers; each step's H2D and D2H inside the timed region, "
                             "overlapping the neighbouring steps' kernels (two copy streams, two slots)"},
@@ -620,6 +620,39 @@ def unmasked_pair_count(torch, kv_idx, kv_cnt, tile_q, block_k):
     ramp = torch.where(lo <= hi, (lo + hi) * (hi - lo + 1) // 2, torch.zeros_like(a))
     flat = block_k * (a + tile_q - torch.maximum(a, torch.full_like(a, block_k))).clamp(min=0)
     return float(((ramp + flat) * valid).sum().item())
+
+
+def path_rooflines(spec, score_ms, select_ms, peaks):
+    """Score and selection against their rooflines, from the workload's shape.
+
+    Score (pool + score launches): 2 * d * tile_q flops per (b, h, tile, causal block j <= J_t),
+    the algorithmic count (the bf16 hi/lo split executes twice that), against the sustained
+    tensor peak; and its compulsory bytes (Q and K read, the causal scores written) against HBM.
+    Selection (rank + gate + finalize): the candidate scores j < f_lo(t) read and kv_idx
+    written, against HBM."""
+    n_qt = spec.N // spec.tile_q
+    causal = sum(((t + 1) * spec.tile_q - 1) // spec.block_k + 1 for t in range(n_qt))
+    cand = sum((t * spec.tile_q) // spec.block_k for t in range(n_qt))
+    heads = spec.B * spec.Hq
+    W = min(spec.rho * max(spec.k_first, spec.k_last), spec.N // spec.block_k)
+    score_flop = 2.0 * spec.d * spec.tile_q * causal * heads
+    score_bytes = (heads * spec.N * spec.d * 2 + spec.B * spec.Hkv * spec.N * spec.d * 2
+                   + heads * causal * 4)
+    sel_bytes = heads * cand * 4 + heads * n_qt * W * 4
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    sc_tflops = score_flop / (score_ms * 1e-3) / 1e12
+    sc_gbps = score_bytes / (score_ms * 1e-3) / 1e9
+    sel_gbps = sel_bytes / (select_ms * 1e-3) / 1e9
+    return {
+        "score": {"ms": score_ms, "algorithmic_tflop": score_flop / 1e12, "tflops": sc_tflops,
+                  "frac_tensor_sustained": sc_tflops / sustained,
+                  "executed_frac_tensor_sustained": 2.0 * sc_tflops / sustained,
+                  "bytes": score_bytes, "GBps": sc_gbps, "frac_hbm": sc_gbps / hbm,
+                  "note": "pool + score launches; hi/lo split executes 2x the algorithmic flops"},
+        "select": {"ms": select_ms, "bytes": sel_bytes, "GBps": sel_gbps, "frac_hbm": sel_gbps / hbm,
+                   "note": "rank + gate + finalize; candidate scores read, kv_idx written"},
+    }
 
 
 def _attend_sha():

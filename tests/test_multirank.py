@@ -75,3 +75,23 @@ def test_unmasked_pair_count_matches_brute_force():
                 rows = t * tq + np.arange(tq)[:, None]
                 ref += int((j0 + np.arange(bk)[None, :] <= rows).sum())
         assert got == ref, (tq, bk, got, ref)
+
+
+def test_path_rooflines_closed_forms():
+    """The bench's score and selection work counts against closed forms: with 128-row tiles
+    and 64-key blocks, tile t sees 2t + 2 causal blocks and ranks 2t candidates."""
+    import bench as B
+    from block_sparse_causal_bsa_b200 import synthetic as S
+    spec = S.WORKLOADS[B.WORKLOAD]
+    assert (spec.tile_q, spec.block_k) == (128, 64)
+    n_qt, heads = spec.N // 128, spec.B * spec.Hq
+    r = B.path_rooflines(spec, 2.0, 0.5, {"bf16_tflops_sustained": 1000.0, "hbm_gbs": 5000.0})
+    flop = 2 * spec.d * 128 * heads * n_qt * (n_qt + 1)
+    assert r["score"]["algorithmic_tflop"] == pytest.approx(flop / 1e12)
+    assert r["score"]["tflops"] == pytest.approx(flop / 2e-3 / 1e12)
+    assert r["score"]["frac_tensor_sustained"] == pytest.approx(flop / 2e-3 / 1e12 / 1000.0)
+    q_k = (heads + spec.B * spec.Hkv) * spec.N * spec.d * 2
+    assert r["score"]["bytes"] == q_k + heads * n_qt * (n_qt + 1) * 4
+    W = min(spec.rho * spec.k_first, spec.N // 64)
+    assert r["select"]["bytes"] == heads * n_qt * (n_qt - 1) * 4 + heads * n_qt * W * 4
+    assert r["select"]["frac_hbm"] == pytest.approx(r["select"]["bytes"] / 0.5e-3 / 1e9 / 5000.0)
