@@ -76,9 +76,9 @@ struct RadixSel {
   int take_eq;     // how many keys equal to v (lowest indices first) are inside the top r+1
 };
 
-// Key of the (r+1)-th largest among keys[0..n), n >= r+1. Digits of 8 bits, starting
-// below the bits every key of the row shares (so the first histogram spreads out).
-__device__ RadixSel warp_radix_select(const uint32_t* keys, int n, int r, uint32_t kmin, uint32_t kmax,
+// Key of the (r+1)-th largest among the keys of s[0..n), n >= r+1. Digits of 8 bits,
+// starting below the bits every key of the row shares (so the first histogram spreads out).
+__device__ RadixSel warp_radix_select(const float* s, int n, int r, uint32_t kmin, uint32_t kmax,
                                       uint32_t* hist, int lane) {
   int want = r + 1;
   if (kmin == kmax) return {kmax, want};
@@ -94,7 +94,7 @@ __device__ RadixSel warp_radix_select(const uint32_t* keys, int n, int r, uint32
     for (int k = 0; k < 8; ++k) hist[lane * 8 + k] = 0u;
     __syncwarp();
     for (int i = lane; i < n; i += 32) {
-      const uint32_t u = keys[i];
+      const uint32_t u = score_key(__ldg(s + i));
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
     }
     __syncwarp();
@@ -161,21 +161,22 @@ __device__ __forceinline__ float cut_sigma(float s0, float a, float b) {
   return (den == 0.0f) ? 0.0f : __fdiv_rn(num, den);
 }
 
-// Radix path for one row whose keys are in keys[0..n). Writes the top-M list with
-// the top-m flag to out and returns sigma (1 when the tile has no cut).
-__device__ float rank_row_radix(const uint32_t* keys, uint32_t* hist, int n, const TileSlots& sl,
-                                const float* s, int32_t* out, int lane) {
+// Radix path for the row s[0..n), ranked on order-preserving keys. Writes the top-M list
+// with the top-m flag to out and returns sigma (1 when the tile has no cut).
+__device__ float rank_row_radix(uint32_t* hist, int n, const TileSlots& sl, const float* s,
+                                int32_t* out, int lane) {
   uint32_t kmax = 0u, kmin = 0xffffffffu;
   for (int i = lane; i < n; i += 32) {
-    kmax = max(kmax, keys[i]);
-    kmin = min(kmin, keys[i]);
+    const uint32_t u = score_key(__ldg(s + i));
+    kmax = max(kmax, u);
+    kmin = min(kmin, u);
   }
   kmax = warp_max_u32(kmax);
   kmin = warp_min_u32(kmin);
   const int m = sl.m, M = sl.M;
   RadixSel selm{0u, 0}, selM{0u, 0};
-  if (m > 0 && m < n) selm = warp_radix_select(keys, n, m - 1, kmin, kmax, hist, lane);
-  if (M > m && M < n) selM = warp_radix_select(keys, n, M - 1, kmin, kmax, hist, lane);
+  if (m > 0 && m < n) selm = warp_radix_select(s, n, m - 1, kmin, kmax, hist, lane);
+  if (M > m && M < n) selM = warp_radix_select(s, n, M - 1, kmin, kmax, hist, lane);
   else if (M == m) selM = selm;
   const bool all_m = m >= n, all_M = M >= n;
 
@@ -188,7 +189,7 @@ __device__ float rank_row_radix(const uint32_t* keys, uint32_t* hist, int n, con
   for (int b0 = 0; b0 < n; b0 += 32) {
     const int i = b0 + lane;
     const bool live = i < n;
-    const uint32_t u = live ? keys[i] : 0u;
+    const uint32_t u = live ? score_key(__ldg(s + i)) : 0u;
     const bool e_m = live && !all_m && m > 0 && u == selm.v;
     const unsigned bal_m = __ballot_sync(0xffffffffu, e_m);
     const int r_m = eq_m + __popc(bal_m & lt);
@@ -239,28 +240,53 @@ struct BucketMap {
   }
 };
 
-__host__ __device__ inline int rank_slice_words(int n_kb) {
-  return ((n_kb + 3) & ~3) + 512 + 3 * kListCap;
+// Per-warp shared-memory slice (words): histogram, bucket starts, the list, its scores,
+// and the list regrouped by bucket (scores, positions). The row itself is not staged: each
+// pass reads it from global memory (the second and third passes hit L2), which keeps the
+// slice small and lets ~36 warps run per SM.
+constexpr int kRankSliceWords = 512 + 4 * kListCap;
+constexpr int kRankWarps = 4;                // rows (warps) per CTA
+
+// Chunk c of a row holds its elements 4c..4c+3; those at or past n read as 0 (callers
+// mask them). A chunk is one 16-byte load when the row is 16-byte aligned and the chunk
+// lies wholly inside [0, n); otherwise its elements are loaded one by one.
+struct RowChunks {
+  const float* s;
+  int n;
+  bool al;
+  __device__ __forceinline__ float4 operator()(int c) const {
+    const int i0 = 4 * c;
+    if (al && i0 + 3 < n) return __ldg(reinterpret_cast<const float4*>(s) + c);
+    float4 v;
+    v.x = i0 < n ? __ldg(s + i0) : 0.f;
+    v.y = i0 + 1 < n ? __ldg(s + i0 + 1) : 0.f;
+    v.z = i0 + 2 < n ? __ldg(s + i0 + 2) : 0.f;
+    v.w = i0 + 3 < n ? __ldg(s + i0 + 3) : 0.f;
+    return v;
+  }
+};
+
+__device__ __forceinline__ float f4_at(const float4& v, int j) {
+  return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
 
 // Writes, per row, the top-M candidates (M = expanded slots) in ascending block
 // order with kInTopM set on the top-m ones (m = base slots; top-m is a prefix of
 // the same ranking, so it is a subset), and sigma from ranks 0, m-1, m.
-__global__ void __launch_bounds__(256) select_rank_kernel(
+__global__ void __launch_bounds__(kRankWarps * 32, 8) select_rank_kernel(
     const float* __restrict__ scores, int rows_bh, int n_qt, int n_kb, int tile_q, int block_k,
     int k_first, int k_last, int rho, int R, int32_t* __restrict__ ranked, float* __restrict__ sigma,
     int32_t* dev_status) {
   extern __shared__ __align__(16) uint32_t wsm[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int wpc = blockDim.x / 32;
-  const int bh = blockIdx.y * wpc + warp;
+  const int bh = blockIdx.y * kRankWarps + warp;
   if (bh >= rows_bh) return;
   const int t = n_qt - 1 - (int)blockIdx.x;          // longest rows first
-  float* xs = reinterpret_cast<float*>(wsm + (size_t)warp * rank_slice_words(n_kb));
-  uint32_t* hist = reinterpret_cast<uint32_t*>(xs + ((n_kb + 3) & ~3));
+  uint32_t* hist = wsm + (size_t)warp * kRankSliceWords;
   uint32_t* start = hist + 256;
   uint32_t* list = start + 256;                      // block index | bucket << 16, then | rank << 16
-  float* sv = reinterpret_cast<float*>(list + kListCap);   // list regrouped by bucket: scores
+  float* lv = reinterpret_cast<float*>(list + kListCap);    // the list's scores
+  float* sv = lv + kListCap;                         // list regrouped by bucket: scores
   uint32_t* sp = reinterpret_cast<uint32_t*>(sv + kListCap);  // ... list position | block index << 16
   const size_t row = (size_t)bh * n_qt + t;
   const TileSlots sl = tile_slots(t, n_qt, tile_q, block_k, k_first, k_last, rho);
@@ -271,51 +297,46 @@ __global__ void __launch_bounds__(256) select_rank_kernel(
     if (lane == 0) sigma[row] = 1.0f;
     return;
   }
+  const RowChunks rd{s, n, (reinterpret_cast<uintptr_t>(s) & 15) == 0};
+  const int nc = (n + 3) >> 2;
 
-  // stage the row; its min, max and finiteness
+  // the row's min, max and finiteness (four 16-byte loads per lane in flight)
   float xmin = INFINITY, xmax = -INFINITY;
   bool bad = false;
-  int done = 0;
-  if ((reinterpret_cast<uintptr_t>(s) & 15) == 0) {
-    const float4* s4 = reinterpret_cast<const float4*>(s);
-    float4* x4 = reinterpret_cast<float4*>(xs);
-    const int n4 = n >> 2;
-    for (int c0 = 0; c0 < n4; c0 += 128) {           // four 16-byte loads per lane in flight
-      float4 v[4];
+  for (int c0 = 0; c0 < nc; c0 += 128) {
+    float4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + u * 32 + lane;
-        v[u] = c < n4 ? __ldg(s4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * 32 + lane;
+      v[u] = c < nc ? rd(c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + u * 32 + lane;
-        if (c < n4) {
-          x4[c] = v[u];
-          xmin = fminf(fminf(xmin, v[u].x), fminf(v[u].y, fminf(v[u].z, v[u].w)));
-          xmax = fmaxf(fmaxf(xmax, v[u].x), fmaxf(v[u].y, fmaxf(v[u].z, v[u].w)));
-          bad |= !(isfinite(v[u].x) && isfinite(v[u].y) && isfinite(v[u].z) && isfinite(v[u].w));
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (4 * c + 3 < n) {
+        xmin = fminf(fminf(xmin, v[u].x), fminf(v[u].y, fminf(v[u].z, v[u].w)));
+        xmax = fmaxf(fmaxf(xmax, v[u].x), fmaxf(v[u].y, fmaxf(v[u].z, v[u].w)));
+        bad |= !(isfinite(v[u].x) && isfinite(v[u].y) && isfinite(v[u].z) && isfinite(v[u].w));
+      } else if (c < nc) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (4 * c + j < n) {
+            const float x = f4_at(v[u], j);
+            xmin = fminf(xmin, x);
+            xmax = fmaxf(xmax, x);
+            bad |= !isfinite(x);
+          }
         }
       }
     }
-    done = 4 * n4;
-  }
-  for (int i = done + lane; i < n; i += 32) {
-    const float x = __ldg(s + i);
-    xs[i] = x;
-    xmin = fminf(xmin, x);
-    xmax = fmaxf(xmax, x);
-    bad |= !isfinite(x);
   }
   xmin = warp_min_f32(xmin);
   xmax = warp_max_f32(xmax);
   bad = __any_sync(0xffffffffu, bad);
-  __syncwarp();
 
   const int m = sl.m, M = sl.M;
   const int need = min(n, max(M, m + 1));
   const unsigned lt = (1u << lane) - 1u;
-  const float4* x4 = reinterpret_cast<const float4*>(xs);
   bool radix = bad || !(xmax > xmin);
   float sg = 1.0f;
   int L = 0, bcut = 0;
@@ -325,13 +346,21 @@ __global__ void __launch_bounds__(256) select_rank_kernel(
 #pragma unroll
     for (int k = 0; k < 8; ++k) hist[k * 32 + lane] = 0u;
     __syncwarp();
-    for (int c = lane; 4 * c < n; c += 32) {
-      const float4 v = x4[c];
-      const int i = 4 * c;
-      atomicAdd(&hist[hidx(bk(v.x))], 1u);
-      if (i + 1 < n) atomicAdd(&hist[hidx(bk(v.y))], 1u);
-      if (i + 2 < n) atomicAdd(&hist[hidx(bk(v.z))], 1u);
-      if (i + 3 < n) atomicAdd(&hist[hidx(bk(v.w))], 1u);
+    for (int c0 = 0; c0 < nc; c0 += 128) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        v[u] = c < nc ? rd(c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = 4 * (c0 + u * 32 + lane);
+        if (i < n) atomicAdd(&hist[hidx(bk(v[u].x))], 1u);
+        if (i + 1 < n) atomicAdd(&hist[hidx(bk(v[u].y))], 1u);
+        if (i + 2 < n) atomicAdd(&hist[hidx(bk(v[u].z))], 1u);
+        if (i + 3 < n) atomicAdd(&hist[hidx(bk(v[u].w))], 1u);
+      }
     }
     __syncwarp();
     uint32_t h8[8], ab[8], sum = 0;
@@ -367,32 +396,43 @@ __global__ void __launch_bounds__(256) select_rank_kernel(
     __syncwarp();
   }
   if (!radix) {
-    // the list: every entry in bucket bcut or above, in block order
+    // the list: every entry in bucket bcut or above, in block order, with its score
     int base = 0;
-    for (int c0 = 0; c0 < n; c0 += 128) {
-      const int i0 = c0 + 4 * lane;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i0 < n) v = x4[i0 >> 2];
-      const float vv[4] = {v.x, v.y, v.z, v.w};
-      int bj[4], cnt = 0;
-      bool sj[4];
+    for (int c0 = 0; c0 < nc; c0 += 128) {
+      float4 v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        bj[j] = bk(vv[j]);
-        sj[j] = i0 + j < n && bj[j] >= bcut;
-        cnt += sj[j] ? 1 : 0;
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        v[u] = c < nc ? rd(c) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      int inc = cnt;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, inc, off);
-        if (lane >= off) inc += y;
+      for (int u = 0; u < 4; ++u) {
+        const int i0 = 4 * (c0 + u * 32 + lane);
+        const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        int bj[4], cnt = 0;
+        bool sj[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          bj[j] = bk(vv[j]);
+          sj[j] = i0 + j < n && bj[j] >= bcut;
+          cnt += sj[j] ? 1 : 0;
+        }
+        int inc = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, inc, off);
+          if (lane >= off) inc += y;
+        }
+        int pos = base + inc - cnt;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (sj[j]) {
+            list[pos] = (uint32_t)(i0 + j) | ((uint32_t)bj[j] << 16);
+            lv[pos] = vv[j];
+            ++pos;
+          }
+        base += __shfl_sync(0xffffffffu, inc, 31);
       }
-      int pos = base + inc - cnt;
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (sj[j]) list[pos++] = (uint32_t)(i0 + j) | ((uint32_t)bj[j] << 16);
-      base += __shfl_sync(0xffffffffu, inc, 31);
     }
     __syncwarp();
     // regroup by bucket
@@ -400,7 +440,7 @@ __global__ void __launch_bounds__(256) select_rank_kernel(
       const uint32_t e = list[p];
       const uint32_t idx = e & 0xffffu;
       const uint32_t slot = atomicAdd(&hist[hidx((int)(e >> 16))], 1u);
-      sv[slot] = xs[idx];
+      sv[slot] = lv[p];
       sp[slot] = (uint32_t)p | (idx << 16);
     }
     __syncwarp();
@@ -438,13 +478,10 @@ __global__ void __launch_bounds__(256) select_rank_kernel(
       i_0 = warp_min_i32(i_0);
       i_m1 = warp_min_i32(i_m1);
       i_m = warp_min_i32(i_m);
-      sg = cut_sigma(xs[i_0], xs[i_m1], xs[i_m]);
+      sg = cut_sigma(__ldg(s + i_0), __ldg(s + i_m1), __ldg(s + i_m));
     }
   } else {
-    uint32_t* keys = reinterpret_cast<uint32_t*>(xs);
-    for (int i = lane; i < n; i += 32) keys[i] = score_key(xs[i]);
-    __syncwarp();
-    sg = rank_row_radix(keys, hist, n, sl, s, out, lane);
+    sg = rank_row_radix(hist, n, sl, s, out, lane);
   }
   if (lane == 0) {
     if (bad) {
@@ -455,26 +492,23 @@ __global__ void __launch_bounds__(256) select_rank_kernel(
   }
 }
 
-static int rank_warps_per_cta(int n_kb) {
-  const size_t per_warp = (size_t)rank_slice_words(n_kb) * 4;
-  int w = (int)((112u * 1024u) / per_warp);
-  return w < 1 ? 1 : (w > 8 ? 8 : w);
-}
-
 cudaError_t launch_select_rank(const bsa_shape& s, const bsa_select_params& p, const float* scores,
                                int R, int32_t* ranked, float* sigma, int32_t* dev_status,
                                cudaStream_t st) {
   const int n_qt = s.N / s.tile_q, n_kb = s.N / s.block_k;
-  const int wpc = rank_warps_per_cta(n_kb);
-  const size_t smem = (size_t)wpc * rank_slice_words(n_kb) * 4;
+  const size_t smem = (size_t)kRankWarps * kRankSliceWords * 4;
   const int rows_bh = s.B * s.Hq;
-  dim3 grid(n_qt, (rows_bh + wpc - 1) / wpc);
+  dim3 grid(n_qt, (rows_bh + kRankWarps - 1) / kRankWarps);
   cudaError_t e = cudaFuncSetAttribute(select_rank_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  select_rank_kernel<<<grid, wpc * 32, smem, st>>>(scores, rows_bh, n_qt, n_kb, s.tile_q, s.block_k,
-                                                   p.k_first, p.k_last, p.rho, R, ranked, sigma,
-                                                   dev_status);
+  // occupancy is set by the slices: ask for the largest shared-memory carve-out
+  e = cudaFuncSetAttribute(select_rank_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  select_rank_kernel<<<grid, kRankWarps * 32, smem, st>>>(scores, rows_bh, n_qt, n_kb, s.tile_q,
+                                                         s.block_k, p.k_first, p.k_last, p.rho, R,
+                                                         ranked, sigma, dev_status);
   return cudaGetLastError();
 }
 
