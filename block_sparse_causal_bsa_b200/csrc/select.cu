@@ -49,8 +49,9 @@ __device__ void bitonic_sort(K* a, unsigned n, bool descending) {
 }
 
 // ---------------------------------------------------------------------------
-// Ranking: one warp per (b, h, tile) row; the row's scores are staged in the
-// warp's shared-memory slice.
+// Ranking: one warp per (b, h, tile) row, four rows per CTA. Each pass reads the
+// row's scores from global memory (16-byte loads, four per lane in flight); the
+// warp's shared-memory slice holds only the histogram and the short list.
 //
 // Bucket path. A monotone fp32 map of each score onto 256 equal-width value
 // buckets between the row's min and max (x >= y implies bucket(x) >= bucket(y),
@@ -243,7 +244,7 @@ struct BucketMap {
 // Per-warp shared-memory slice (words): histogram, bucket starts, the list, its scores,
 // and the list regrouped by bucket (scores, positions). The row itself is not staged: each
 // pass reads it from global memory (the second and third passes hit L2), which keeps the
-// slice small and lets ~36 warps run per SM.
+// slice small: eight CTAs (32 warps) per SM, bounded by 64 registers per thread.
 constexpr int kRankSliceWords = 512 + 4 * kListCap;
 constexpr int kRankWarps = 4;                // rows (warps) per CTA
 
