@@ -564,6 +564,47 @@ def test_vs_single_diagonal_returns_own_value():
                                atol=1e-12)
 
 
+def test_vs_random_sets_match_masked_sdpa():
+    """Random vertical columns and slash offsets (with duplicates, out-of-range entries and
+    entries past the counts), two query heads per KV head: the oracle equals torch's fp64
+    scaled_dot_product_attention under the boolean mask (j <= i and j a column) or (i - j an
+    offset), built here pair by pair; its lse equals the masked logsumexp, and exactly the
+    rows with an empty mask row come out 0 / -inf."""
+    rng = np.random.default_rng(33)
+    B, Hq, Hkv, N, d = 1, 4, 2, 96, 16
+    Q = S.f32_to_bf16_bits(rng.standard_normal((B, Hq, N, d)).astype(np.float32))
+    K = S.f32_to_bf16_bits(rng.standard_normal((B, Hkv, N, d)).astype(np.float32))
+    V = S.f32_to_bf16_bits(rng.standard_normal((B, Hkv, N, d)).astype(np.float32))
+    Wv, Ws = 12, 9
+    v_idx = rng.integers(-5, N + 5, size=(B, Hq, Wv)).astype(np.int32)
+    s_off = rng.integers(-3, N + 3, size=(B, Hq, Ws)).astype(np.int32)
+    v_idx[0, 0, :3] = [40, 40, 7]                      # duplicates count once
+    s_off[0, 0, :2] = [5, 5]
+    v_cnt = np.array([[Wv, 7, 0, 12]], np.int32)
+    s_cnt = np.array([[Ws, 0, 4, 9]], np.int32)
+    scale = 0.3
+    o, lse = O.attend_vs(Q, K, V, v_idx, v_cnt, s_off, s_cnt, scale)
+    for h in range(Hq):
+        cols = {int(j) for j in v_idx[0, h, :v_cnt[0, h]] if 0 <= j < N}
+        offs = {int(x) for x in s_off[0, h, :s_cnt[0, h]] if 0 <= x < N}
+        mask = np.zeros((N, N), bool)
+        for i in range(N):
+            for j in range(i + 1):
+                mask[i, j] = j in cols or (i - j) in offs
+        q = torch.from_numpy(O.widen(Q[0, h]))
+        k = torch.from_numpy(O.widen(K[0, h // 2]))
+        v = torch.from_numpy(O.widen(V[0, h // 2]))
+        m = torch.from_numpy(mask)
+        live = mask.any(axis=1)
+        ref = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None], attn_mask=m[None],
+                                                               scale=scale)[0].numpy()
+        np.testing.assert_allclose(o[0, h, live], ref[live], rtol=0, atol=1e-12)
+        lg = (scale * (q @ k.T)).masked_fill(~m, float("-inf"))
+        np.testing.assert_allclose(lse[0, h, live], torch.logsumexp(lg, dim=1).numpy()[live], rtol=0, atol=1e-12)
+        assert not o[0, h, ~live].any() and np.isneginf(lse[0, h, ~live]).all()
+        assert live.sum() > N // 4
+
+
 def test_vs_key_sets_and_empty_rows():
     assert list(O.vs_keys(10, [0, 3, 11, 40], [0, 2, 10, 20])) == [0, 3, 8, 10]
     assert list(O.vs_keys(1, [5], [4])) == []
