@@ -69,7 +69,7 @@ cudaError_t launch_attend_tc(const bsa_shape& s, const void* q, const void* k, c
                              void* out, float* lse, int32_t* dev_status, cudaStream_t st);
 
 // Limits of this build (checked on the host).
-constexpr int kMaxCandidates = 8192;     // n_kb for the in-shared-memory ranking sort
+constexpr int kMaxCandidates = 8192;     // n_kb limit of the selection (the range its tests cover)
 constexpr int kMaxGateTiles = 16384;     // B * n_qt for the single-CTA gate sort
 constexpr int kMaxProbe = 64;
 constexpr int kMaxGroup = 8;             // Hq / Hkv in decode

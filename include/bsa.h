@@ -192,7 +192,9 @@ size_t bsa_select_workspace_bytes(const bsa_shape* shape, const bsa_select_param
  *   sigma_bar[B,n_qt] fp32 or NULL: fp32 head sum in head order, / Hq ([UGS] step 4).
  *   trigger  [B,n_qt] uint8 or NULL: cut tile and sigma_bar < theta (strict).
  *   theta    device fp32 scalar or NULL (NaN when undefined).
- *   dev_status device int32 or NULL: BSA_DEV_BAD_SCORE on a non-finite candidate. */
+ *   dev_status device int32 or NULL: BSA_DEV_BAD_SCORE on a non-finite candidate.
+ * Limits: n_kb <= 8192 and B * n_qt <= 16384 (the gate sorts one layer's tiles in one
+ * CTA); beyond them BSA_ERR_UNSUPPORTED and nothing is launched. */
 bsa_status bsa_select(const bsa_shape* shape, const bsa_select_params* params,
                       const float* scores, int32_t* kv_idx, int32_t* kv_cnt,
                       float* sigma, float* sigma_bar, uint8_t* trigger, float* theta,

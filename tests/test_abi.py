@@ -105,7 +105,7 @@ def test_bad_select_params_rejected(kf, kl, rho, q):
 
 def test_select_size_limits():
     L = bb.lib()
-    s = _shape(N=64 * 16384)      # more key blocks than the in-shared-memory sort takes
+    s = _shape(N=64 * 16384)      # more key blocks than the selection supports (8192)
     p = bb.SelectParams(8, 8, 1, 0.25, 0.0)
     assert L.bsa_select(ctypes.byref(s), ctypes.byref(p), 16, 16, 16, None, None, None, None, None,
                         256, 1 << 40, None) == bb.BSA_ERR_UNSUPPORTED
