@@ -46,8 +46,12 @@ block level (the block's mean value vector for V_j, natural log, weight beta,
 no 1/sqrt(d) on the score); the K-min/K-max score is the tile max of
 sum_c max(q_c kmin_c, q_c kmax_c); a vertical-slash row attends to the union,
 each key once, of its vertical columns j <= i and the keys i - o of its slash
-offsets; a decode over a block list visits the list in order and never tests
-its first entry.
+offsets; a decode over a block list visits the list in order, skips entries
+outside the cache (they are not visit steps) and never tests its first visit.
+
+bf16 inputs: ``widen`` reads a uint16 array as bf16 bit patterns (the upper
+half of a float32), exact in fp64; it is pinned over all 65,536 patterns
+against torch's own bfloat16 type and against hand-computed values.
 
 Parity status: every function below is pinned by CPU tests against closed
 forms, library routines (torch scaled_dot_product_attention, numpy.quantile)
@@ -552,6 +556,15 @@ def decode(q, Kc, Vc, block_kv, scale, tau, phi, patience, probe_dims, enable=Tr
     return O, used, traces
 
 
+def decode_visit_steps(blocks: Sequence[int], n_blocks: int) -> list:
+    """The visit sequence of a decode block list: its entries in list order, with
+    every entry outside [0, n_blocks) skipped. A skipped entry is not a visit step
+    (it is neither streamed nor tested); the library reports it as a bad index.
+    [ART, 2.4] only fixes that the traversal order may change; what an index
+    outside the cache means is the library's reading: nothing to visit."""
+    return [int(j) for j in blocks if 0 <= int(j) < n_blocks]
+
+
 def decode_group_list(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, block_kv: int, scale: float,
                       blocks: Sequence[int], tau: float, phi: float, patience: int,
                       probe_dims: np.ndarray, enable: bool = True):
@@ -559,16 +572,17 @@ def decode_group_list(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, block_kv: i
     the result of a full pass does not depend on the order, so a selector's blocks
     may be visited first block first, then most important or most recent first).
 
-    After visit step t the normalised partial output O^(t) of each head is the
-    softmax over all keys of blocks[0..t] applied to V (fp64); the probe, the
-    stability test and the stop rule are those of ``decode_group`` with the visit
-    step in place of the block number (the first listed block is never tested).
-    An empty list gives O = 0 and blocks_used = 0. Returns (O [G, d] fp64,
-    blocks_used, trace [steps used, n_probe] fp32).
+    The visit steps are ``decode_visit_steps(blocks, L // block_kv)``: entries
+    outside the cache are skipped. After visit step t the normalised partial output
+    O^(t) of each head is the softmax over all keys of the first t+1 visited blocks
+    applied to V (fp64); the probe, the stability test and the stop rule are those
+    of ``decode_group`` with the visit step in place of the block number (the first
+    visited block is never tested). No visit step gives O = 0 and blocks_used = 0.
+    Returns (O [G, d] fp64, blocks_used, trace [steps used, n_probe] fp32).
     """
     qf, Kf, Vf = widen(q), widen(Kc), widen(Vc)
     G, d = qf.shape
-    blocks = [int(j) for j in blocks]
+    blocks = decode_visit_steps(blocks, Kf.shape[0] // block_kv)
     n = len(blocks)
     if n == 0:
         return np.zeros((G, d)), 0, np.zeros((0, len(probe_dims)), np.float32)
@@ -588,8 +602,9 @@ def decode_group_list(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, block_kv: i
 def decode_list(q, Kc, Vc, block_kv, scale, block_list, list_cnt, tau, phi, patience, probe_dims,
                 enable=True):
     """q [B,Hq,d], caches [B,Hkv,L,d], block_list [B,Hkv,W] int (visit order, the
-    first list_cnt[b,g] entries used) -> (O [B,Hq,d] fp64, blocks_used [B,Hkv],
-    traces {(b, g): trace})."""
+    first list_cnt[b,g] entries used; a count outside [0, W] is clamped to it, and
+    entries outside the cache are skipped by ``decode_group_list``) ->
+    (O [B,Hq,d] fp64, blocks_used [B,Hkv], traces {(b, g): trace})."""
     B, Hq, d = q.shape
     Hkv = Kc.shape[1]
     G = Hq // Hkv
@@ -598,7 +613,8 @@ def decode_list(q, Kc, Vc, block_kv, scale, block_list, list_cnt, tau, phi, pati
     traces = {}
     for b in range(B):
         for g in range(Hkv):
-            lst = np.asarray(block_list[b, g][:int(list_cnt[b, g])])
+            W = block_list.shape[-1]
+            lst = np.asarray(block_list[b, g][:min(max(int(list_cnt[b, g]), 0), W)])
             o, u, tr = decode_group_list(q[b, g * G:(g + 1) * G], Kc[b, g], Vc[b, g], block_kv,
                                          scale, lst, tau, phi, patience, probe_dims, enable)
             O[b, g * G:(g + 1) * G] = o

@@ -29,7 +29,9 @@ def check_scores(gpu: np.ndarray, ref: np.ndarray):
     a = np.where(fin, np.abs(ref.astype(np.float64)), 0.0)
     rbar = a.sum(-1) / np.maximum(fin.sum(-1), 1)
     tol = SCORE_RTOL * np.maximum(a, rbar[..., None])
-    err = np.where(fin, np.abs(gpu.astype(np.float64) - ref), 0.0)
+    diff = np.zeros(ref.shape, np.float64)
+    diff[fin] = np.abs(gpu[fin].astype(np.float64) - ref[fin].astype(np.float64))
+    err = diff
     bad = err > tol
     assert not bad.any(), f"{bad.sum()} score entries off; worst rel {(err / np.maximum(tol, 1e-30)).max() * SCORE_RTOL:.3e}"
     return float((err / np.maximum(tol / SCORE_RTOL, 1e-30)).max())

@@ -39,19 +39,23 @@ def _run(spec, seed, lists, cnt, tau, phi, patience, enable=True, expect_status=
     agree = 0
     for b in range(spec.B):
         for g in range(spec.Hkv):
-            row = lists[b, g, :max(0, min(int(cnt[b, g]), lists.shape[-1]))]
-            valid = [int(j) for j in row if 0 <= j < nb]          # the visit sequence
+            raw = lists[b, g, :max(0, min(int(cnt[b, g]), lists.shape[-1]))]   # the list as given
+            steps = O.decode_visit_steps(raw, nb)        # the oracle's visit sequence
             u = int(used[b, g])
-            n = len(valid)
+            n = len(steps)
             exp = (O.termination_block(trace[b, g], tau, phi, patience, n_blocks=n)
                    if enable and n > 0 else n)
             assert u == exp, (b, g, u, exp)
             qg = q[b, g * G:(g + 1) * G]
-            o_ref, _, _ = O.decode_group_list(qg, k[b, g], v[b, g], spec.block_kv, scale,
-                                              valid[:u], tau, phi, patience, dims, enable=False)
+            # output after the GPU's u visit steps: the shortest prefix of the raw list
+            # holding u visit steps, through the oracle (which skips the bad entries itself)
+            pre = next(i for i in range(len(raw) + 1) if len(O.decode_visit_steps(raw[:i], nb)) == u)
+            o_ref, u_pre, _ = O.decode_group_list(qg, k[b, g], v[b, g], spec.block_kv, scale,
+                                                  raw[:pre], tau, phi, patience, dims, enable=False)
+            assert u_pre == u
             check_attend(go[b, g * G:(g + 1) * G], o_ref)
             _, u_ref, tr_ref = O.decode_group_list(qg, k[b, g], v[b, g], spec.block_kv, scale,
-                                                   valid, tau, phi, patience, dims, enable=enable)
+                                                   raw, tau, phi, patience, dims, enable=enable)
             agree += int(u_ref == u)
             m = min(u, u_ref)
             np.testing.assert_allclose(trace[b, g, :m], tr_ref[:m], atol=2e-3)

@@ -5,9 +5,11 @@ The scores are drawn here, seeded, per row from one of six structures that
 stress the exact ranking: plain Gaussian values, a handful of levels (long runs
 of ties broken by block index), a constant row, values a few ulps apart (keys
 that differ only in their lowest bits), mixed signs with signed zeros, and
-magnitudes from 1e-30 to 1e30. Row widths cover every ranking kernel: 512, 1024
-and 2048 candidate blocks (keys held in registers) and 4096 (keys in shared
-memory).
+magnitudes from 1e-30 to 1e30. Together they reach both ranking paths of the
+selection kernel: the value-bucket path (short candidate lists ranked by
+pairwise counts) and its exact radix fallback (constant rows, long tie runs,
+buckets or lists too large for the short path). Row widths run from 512 to 4096
+candidate blocks.
 """
 import numpy as np
 import pytest

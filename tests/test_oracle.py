@@ -769,3 +769,105 @@ def test_gated_workload_near_tie_fraction():
                 near += float(s[o[m - 1]]) - float(s[o[m]]) < 1e-3
                 tot += 1
     assert 0.15 <= near / tot <= 0.25, near / tot
+
+
+# ---------------------------------------------------------------------------
+# bf16 storage: the oracle's widening and the generator's rounding, each against
+# an implementation that shares nothing with it
+
+def _bf16_value(bits: int) -> float:
+    """A bf16 bit pattern's value from its fields (sign, 8-bit exponent, 7-bit
+    fraction), written out for a handful of fixed cases."""
+    sign = -1.0 if bits & 0x8000 else 1.0
+    e, f = (bits >> 7) & 0xFF, bits & 0x7F
+    if e == 0xFF:
+        return sign * math.inf
+    if e == 0:
+        return sign * f * 2.0 ** -133               # subnormal: f * 2^(1 - 127 - 7)
+    return sign * (1.0 + f / 128.0) * 2.0 ** (e - 127)
+
+
+def test_widen_bf16_every_pattern_matches_torch():
+    """Every non-NaN bf16 pattern widens to the value torch's bfloat16 holds."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    nan = ((bits & 0x7F80) == 0x7F80) & ((bits & 0x7F) != 0)
+    bits = bits[~nan]
+    ours = O.widen(bits)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
+    assert ours.dtype == np.float64
+    np.testing.assert_array_equal(ours, ref)
+    # the sign of zero survives too
+    assert np.array_equal(np.signbit(ours), np.signbit(ref))
+
+
+@pytest.mark.parametrize("bits", [0x0000, 0x8000, 0x0001, 0x8001, 0x007F, 0x0080, 0x3F80, 0xBF80,
+                                  0x4000, 0xC000, 0x3F81, 0x4049, 0x7F7F, 0xFF7F, 0x7F80, 0xFF80])
+def test_widen_bf16_special_values(bits):
+    """+-0, the smallest and largest subnormals, the smallest normal, +-1, +-2, 1 + 2^-7,
+    3.140625, the largest finite values and the infinities, from their fields."""
+    got = float(O.widen(np.array([bits], np.uint16))[0])
+    exp = _bf16_value(bits)
+    assert got == exp and math.copysign(1.0, got) == math.copysign(1.0, exp)
+
+
+def test_generator_rounding_matches_torch():
+    """The generator's float32 -> bf16 rounding (nearest, ties to even) against
+    torch's conversion: random values over the whole exponent range, subnormals,
+    values that round up to infinity, and exact ties with even and odd upper halves."""
+    rng = np.random.default_rng(11)
+    u = rng.integers(0, 1 << 32, size=200_000, dtype=np.uint64).astype(np.uint32)
+    x = u.view(np.float32)
+    x = x[np.isfinite(x)]
+    hi = rng.integers(0, 1 << 16, size=4096, dtype=np.uint32)
+    hi = hi[((hi & 0x7F80) != 0x7F80)]
+    ties = ((hi << 16) | 0x8000).astype(np.uint32).view(np.float32)           # exactly halfway
+    near = np.concatenate([((hi << 16) | 0x7FFF), ((hi << 16) | 0x8001)]).astype(np.uint32).view(np.float32)
+    extra = np.array([0.0, -0.0, 1e-45, -1e-45, 1.17549435e-38, 3.4028235e38, -3.4028235e38,
+                      np.float32(np.inf), -np.float32(np.inf), 1.0, -1.0, 1.00390625, 1.01171875],
+                     np.float32)
+    for arr in (x, ties, near, extra):
+        ours = S.f32_to_bf16_bits(arr)
+        ref = torch.from_numpy(np.ascontiguousarray(arr)).to(torch.bfloat16).view(torch.int16).numpy()
+        np.testing.assert_array_equal(ours.view(np.int16), ref)
+    # ties go to the even neighbour: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7
+    assert S.f32_to_bf16_bits(np.array([1.00390625], np.float32))[0] == 0x3F80
+    assert S.f32_to_bf16_bits(np.array([1.01171875], np.float32))[0] == 0x3F82
+
+
+def test_decode_list_skips_entries_outside_the_cache():
+    """Entries outside [0, L/block_kv) are not visit steps: a list holding -7, one
+    past the last block and valid blocks gives what the valid blocks alone give,
+    and a full pass is textbook attention over exactly those blocks."""
+    q, Kc, Vc = _decode_case()
+    dims = S.default_probe_dims(32)
+    nb = Kc.shape[0] // 128
+    raw = [3, -7, 11, nb, 0, nb + 40, 6]
+    valid = [3, 11, 0, 6]
+    assert O.decode_visit_steps(raw, nb) == valid
+    for tau, phi in [(0.0, 0.0), (1e-3, 1e-4), (np.inf, np.inf)]:
+        a = O.decode_group_list(q, Kc, Vc, 128, 0.125, raw, tau, phi, 1, dims)
+        b = O.decode_group_list(q, Kc, Vc, 128, 0.125, valid, tau, phi, 1, dims)
+        assert a[1] == b[1]
+        np.testing.assert_array_equal(a[0], b[0])
+        np.testing.assert_array_equal(a[2], b[2])
+    o, used, _ = O.decode_group_list(q, Kc, Vc, 128, 0.125, raw, 0.0, 0.0, 1, dims)
+    assert used == 4
+    np.testing.assert_allclose(o, _sdpa_over_blocks(q, Kc, Vc, valid, 0.125), atol=1e-12)
+    # only bad entries: nothing to visit
+    o, used, tr = O.decode_group_list(q, Kc, Vc, 128, 0.125, [-1, nb], 0.0, 0.0, 1, dims)
+    assert used == 0 and tr.shape == (0, 32) and not o.any()
+
+
+def test_decode_list_counts_are_clamped():
+    """list_cnt outside [0, W] is clamped: a negative count visits nothing, a count
+    above the width visits the whole row."""
+    q, Kc, Vc = _decode_case()
+    dims = S.default_probe_dims(32)
+    qq = np.stack([np.tile(q, (1, 1))])                   # [1, G, d]
+    lists = np.array([[[0, 5, 9]]], np.int32)
+    _, used, _ = O.decode_list(qq, Kc[None, None], Vc[None, None], 128, 0.125, lists,
+                               np.array([[-3]]), 0.0, 0.0, 1, dims)
+    assert used[0, 0] == 0
+    _, used, _ = O.decode_list(qq, Kc[None, None], Vc[None, None], 128, 0.125, lists,
+                               np.array([[17]]), 0.0, 0.0, 1, dims)
+    assert used[0, 0] == 3
