@@ -233,7 +233,8 @@ def cpu_baseline(spec, seed, target_s=15.0):
     dt, _ = cpu_sample(spec, seed, n, rng_seed=3, cache=cache)
     n = int(max(16, min(8192, n * target_s / max(dt, 1e-3))))
     dt, fl = cpu_sample(spec, seed, n, cache=cache)
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(),
+            "host_cpus": os.cpu_count(), "kind": "oracle",
             "sample": f"{n} random (b,h,t) tiles of {spec.name}: pooling of their KV groups, "
                       f"scores, ranking+sigma, gate over the sample, sparse attend; "
                       f"{dt:.1f} s, selected-block flops / time"}
@@ -509,10 +510,14 @@ def main_gpu(args):
     for kind, keep in (("recency", 0), ("subset", 64)):
         lh, ch = S.decode_block_lists(dspec, 2006 + 1000 * rank, kind, keep)
         lists[kind] = (torch.from_numpy(lh).to(dev), torch.from_numpy(ch).to(dev), lh.shape[-1])
-    runs = (("terminated", 1, None), ("full_scan", 0, None), ("listed_recency", 1, "recency"),
-            ("listed_subset64", 1, "subset"))
-    for label, enable, lk in runs:
-        dp = bb.DecodeParams(dspec.tau, dspec.phi, dspec.patience, enable, len(dims), cdims)
+    # detector_on: the stability test runs after every block but can never pass (tau = phi = 0),
+    # so the scan is as long as full_scan (test off); their difference is the detector's cost
+    runs = (("terminated", 1, None, dspec.tau, dspec.phi), ("full_scan", 0, None, dspec.tau, dspec.phi),
+            ("detector_on", 1, None, 0.0, 0.0),
+            ("listed_recency", 1, "recency", dspec.tau, dspec.phi),
+            ("listed_subset64", 1, "subset", dspec.tau, dspec.phi))
+    for label, enable, lk, tau_, phi_ in runs:
+        dp = bb.DecodeParams(tau_, phi_, dspec.patience, enable, len(dims), cdims)
 
         def run_decode():
             if lk is None:
@@ -543,6 +548,10 @@ def main_gpu(args):
         dec[label] = {"ms": ms, "blocks_used": blocks, "bytes": byts, "GBps": byts / ms / 1e6}
     peaks, peak_kind = _peaks()
     dec["hbm_frac_full_scan"] = dec["full_scan"]["GBps"] / peaks["hbm_gbs"]
+    dec["hbm_frac_terminated"] = dec["terminated"]["GBps"] / peaks["hbm_gbs"]
+    if dec["detector_on"]["blocks_used"] != dec["full_scan"]["blocks_used"]:
+        raise RuntimeError("decode with tau = phi = 0 stopped early")
+    dec["detector_overhead_pct"] = 100.0 * (dec["detector_on"]["ms"] / dec["full_scan"]["ms"] - 1.0)
     dec["mean_blocks_used"] = dec["terminated"]["blocks_used"] / (dspec.B * dspec.Hkv)
     dec["blocks_total"] = dspec.L // dspec.block_kv
     dec["peak_note"] = f"{peak_kind} HBM {peaks['hbm_gbs']} GB/s"
@@ -553,6 +562,7 @@ def main_gpu(args):
     if rank == 0:
         sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        sm_max = float(clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0))
         achieved = flops / (attend_ms * 1e-3) / 1e12
         achieved_unmasked = 4.0 * d * unmasked_pairs / (attend_ms * 1e-3) / 1e12
         traffic = None
@@ -581,16 +591,24 @@ def main_gpu(args):
             "score_backbones_ms": score_kinds,
             "vertical_slash": vs_res,
             "attend_detail": {"frac_of_burst_peak": achieved / burst, "burst_peak": burst,
+                              "frac_of_sustained_peak": achieved / sustained, "sustained_peak": sustained,
                               "frac_of_datasheet_dense": achieved / 2250.0,
                               "unmasked_pair_tflops": achieved_unmasked,
                               "unmasked_pairs": unmasked_pairs,
                               "step_ms_median": float(np.median(per.sum(axis=1))),
                               "attend_ms_median": float(np.median(per[:, 2])),
                               "warm_no_flush": warm},
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained,
-                         "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst,
+                         "unit": "TFLOP/s", "frac": achieved / burst, "traffic": traffic,
                          "kernel": "attend",
-                         "peak_note": f"{peak_kind} sustained dense bf16 (kernel timed inside a step)"},
+                         "frac_of_sustained": achieved / sustained,
+                         "frac_per_clock_of_burst": (achieved / burst) * (sm_max / clocks["sm_mhz"])
+                         if clocks.get("sm_mhz") else None,
+                         "peak_note": f"{peak_kind} burst dense bf16 ({burst}; the timed region lasts "
+                                      f"under a second); frac_of_sustained divides by the "
+                                      f"{sustained} seconds-long figure, frac_per_clock_of_burst "
+                                      f"rescales the achieved rate to {sm_max:.0f} MHz from the "
+                                      f"sampled median SM clock"},
             "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "note": "pinned host buffers; each step's H2D and D2H inside the timed region, "
@@ -687,7 +705,8 @@ def main_reference(args):
            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
            "config": {"workload": WORKLOAD, "sample_tiles_per_step": n_tiles},
-           "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+           "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores,
+                            "host_cpus": os.cpu_count(), "kind": "oracle",
                             "sample": f"{n_tiles} random (b,h,t) tiles per step through the oracle's "
                                       "pool/score/rank/gate/attend"},
            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

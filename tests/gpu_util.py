@@ -49,20 +49,25 @@ def check_selection(g: dict, r: dict):
                           np.array([r["theta"]], np.float32).view(np.uint32))
 
 
-def check_attend(gpu_rows: np.ndarray, ref_rows: np.ndarray):
-    """Attention outputs: max |gpu - ref| / max(1, |ref|) <= 2e-2 and mean |gpu - ref| <= 1e-3.
+def check_attend(gpu_rows: np.ndarray, ref_rows: np.ndarray, lognormal_v: bool = False):
+    """Attention outputs: max |gpu - ref| <= 2e-2 and mean |gpu - ref| <= 1e-3.
 
-    For outputs of magnitude <= 1 this is the plain 2e-2 max-abs bar. Above 1 the
-    bar scales with the output: rounding an exact output to bf16 alone moves it by
-    up to half an ulp, 2^-9 |O| (0.031 at |O| = 8), which the log-normal-V workload
-    reaches, so an absolute bar there would reject a perfectly rounded result."""
+    With lognormal_v (the workload whose value rows have log-normal norms) the max
+    bar scales with the output above 1: max |gpu - ref| / max(1, |ref|) <= 2e-2.
+    Rounding an exact output to bf16 alone moves it by up to half an ulp, 2^-9 |O|
+    (0.031 at |O| = 8), which that workload reaches, so an absolute bar there would
+    reject a perfectly rounded result. Every other workload is held to the plain
+    absolute bar. Returns (max abs error, mean abs error, number of elements that
+    pass only through the scaling)."""
     ref_rows = np.asarray(ref_rows, dtype=np.float64)
     err = np.abs(gpu_rows.astype(np.float64) - ref_rows)
     assert np.isfinite(gpu_rows).all()
     scaled = err / np.maximum(1.0, np.abs(ref_rows))
-    mx, mean = float(scaled.max()), float(err.mean())
-    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, float(err.max()), mean)
-    return float(err.max()), mean
+    n_scaled = int(((err > ATT_MAX_ABS) & (scaled <= ATT_MAX_ABS)).sum())
+    mx = float(scaled.max()) if lognormal_v else float(err.max())
+    mean = float(err.mean())
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, float(err.max()), mean, n_scaled)
+    return float(err.max()), mean, n_scaled
 
 
 def out_rows(t: torch.Tensor) -> np.ndarray:

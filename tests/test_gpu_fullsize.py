@@ -59,11 +59,14 @@ def _full_prefill(name, seed, n_rows=24, n_tiles=12):
               for _ in range(n_tiles)]
     go = out_rows(out)
     scale = 1.0 / math.sqrt(spec.d)
+    lognormal = spec.structure == "lognormal_v"
+    n_scaled = 0
     for b, h, t in tiles:
         r0 = t * spec.tile_q
         ro, _ = O.attend_tile(q[b, h, r0:r0 + spec.tile_q], k[b, h // G], v[b, h // G],
                               ref_sel["kv_idx"][b, h, t], r0, spec.block_k, scale)
-        check_attend(go[b, h, r0:r0 + spec.tile_q], ro)
+        n_scaled += check_attend(go[b, h, r0:r0 + spec.tile_q], ro, lognormal_v=lognormal)[2]
+    print(f"{name}: {n_scaled} output elements pass only through the max(1, |O|) scaling")
     return spec, ref_sel
 
 

@@ -45,12 +45,14 @@ def _run_prefill(spec, seed, k_first=None, k_last=None, tiles=None):
     scale = 1.0 / math.sqrt(spec.d)
     ro, _ = O.attend(q, k, v, ref_sel["kv_idx"], spec.tile_q, spec.block_k, scale, tiles=tiles)
     go = out_rows(out)
+    lognormal = spec.structure == "lognormal_v"
     if tiles is None:
-        check_attend(go, ro)
+        check_attend(go, ro, lognormal_v=lognormal)
     else:
         for b, h, t in tiles:
             r0 = t * spec.tile_q
-            check_attend(go[b, h, r0:r0 + spec.tile_q], ro[b, h, r0:r0 + spec.tile_q])
+            check_attend(go[b, h, r0:r0 + spec.tile_q], ro[b, h, r0:r0 + spec.tile_q],
+                         lognormal_v=lognormal)
     return sel, ref_sel
 
 

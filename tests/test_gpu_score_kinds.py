@@ -39,7 +39,7 @@ def _run(spec, seed, kind, beta=0.0):
                        cfg.gate_quantile)
     check_selection(sel, ref_sel)
     ro, _ = O.attend(q, k, v, ref_sel["kv_idx"], spec.tile_q, spec.block_k, 1 / math.sqrt(spec.d))
-    check_attend(out_rows(out), ro)
+    check_attend(out_rows(out), ro, lognormal_v=spec.structure == "lognormal_v")
     return g, ref_sel
 
 
