@@ -310,22 +310,36 @@ def main_gpu(args):
     ws_s = torch.empty(ws_s_n, dtype=torch.uint8, device=dev)
     ws_l_n = bb.bsa_select_workspace_bytes(shape, prm)
     ws_l = torch.empty(ws_l_n, dtype=torch.uint8, device=dev)
+    ws_f_n = bb.bsa_score_select_workspace_bytes(shape, bb.BSA_SCORE_MEAN, prm)
+    ws_f = torch.empty(ws_f_n, dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     scale = 1.0 / math.sqrt(d)
 
     def step(q_, k_, v_, out_, ev=None):
+        # scores and selection in one call (the ranking runs inside the score kernel; the
+        # scores are not written out), then the sparse attend
         if ev:
             ev[0].record(stream)
-        bb.bsa_score(shape, bb.BSA_SCORE_MEAN, q_, k_, None, scores, st_score, ws_s, ws_s_n, sh)
+        bb.bsa_score_select(shape, bb.BSA_SCORE_MEAN, None, prm, q_, k_, None, None, kv_idx, kv_cnt,
+                            None, None, None, theta, st_sel, ws_f, ws_f_n, sh)
+        if ev:
+            ev[1].record(stream)
+        bb.bsa_attend(shape, q_, k_, v_, kv_idx, kv_cnt, W, scale, out_, None, st_att, sh)
+        if ev:
+            ev[2].record(stream)
+
+    def unfused(ev=None):
+        # the same selection through the separate calls: bsa_score writes the scores, bsa_select
+        # reads them back
+        if ev:
+            ev[0].record(stream)
+        bb.bsa_score(shape, bb.BSA_SCORE_MEAN, q, k, None, scores, st_score, ws_s, ws_s_n, sh)
         if ev:
             ev[1].record(stream)
         bb.bsa_select(shape, prm, scores, kv_idx, kv_cnt, None, None, None, theta, st_sel,
                       ws_l, ws_l_n, sh)
         if ev:
             ev[2].record(stream)
-        bb.bsa_attend(shape, q_, k_, v_, kv_idx, kv_cnt, W, scale, out_, None, st_att, sh)
-        if ev:
-            ev[3].record(stream)
 
     for _ in range(args.warmup):
         step(q, k, v, out)
@@ -336,9 +350,9 @@ def main_gpu(args):
     # unmasked (i, j) pairs of the selected blocks (j <= i), for the alternative count: a block
     # wholly below the tile's first row contributes tile_q * block_k pairs, a diagonal block fewer
     unmasked_pairs = unmasked_pair_count(torch, kv_idx, kv_cnt, spec.tile_q, spec.block_k)
-    launches_per_step = 6     # pool, score, select_rank, gate, finalize, attend
+    launches_per_step = 5     # pool, score+rank, gate, finalize, attend
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -347,7 +361,7 @@ def main_gpu(args):
         for i in range(args.steps):
             flush.zero_()
             step(q, k, v, out, evs[i])
-            st_acc.bitwise_or_(st_sel).bitwise_or_(st_att).bitwise_or_(st_score)   # after the events
+            st_acc.bitwise_or_(st_sel).bitwise_or_(st_att)   # after the events
         torch.cuda.synchronize()
         clk.mark(False)
     if int(st_acc.item()) != 0:
@@ -356,18 +370,32 @@ def main_gpu(args):
         dist.barrier()
     torch.cuda.synchronize()
     clocks = clk.summary()
-    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(args.steps)])
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(2)] for i in range(args.steps)])
     step_ms = float(per.sum(axis=1).mean())
-    score_ms, select_ms, attend_ms = (float(x) for x in per.mean(axis=0))
+    score_select_ms, attend_ms = (float(x) for x in per.mean(axis=0))
+    kv_fused = kv_idx.clone()
 
     # warm variant: the same steps without the L2 flush in between
-    wevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(5)]
+    wevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(5)]
     for i in range(5):
         step(q, k, v, out, wevs[i])
     torch.cuda.synchronize()
-    wper = np.array([[wevs[i][j].elapsed_time(wevs[i][j + 1]) for j in range(3)] for i in range(5)])
-    warm = {"step_ms": float(wper.sum(axis=1).mean()), "score_ms": float(wper[:, 0].mean()),
-            "select_ms": float(wper[:, 1].mean()), "attend_ms": float(wper[:, 2].mean())}
+    wper = np.array([[wevs[i][j].elapsed_time(wevs[i][j + 1]) for j in range(2)] for i in range(5)])
+    warm = {"step_ms": float(wper.sum(axis=1).mean()), "score_select_ms": float(wper[:, 0].mean()),
+            "attend_ms": float(wper[:, 1].mean())}
+
+    # the separate calls, timed the same way (cold), for comparison with the fused call
+    uevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(5)]
+    for i in range(5):
+        flush.zero_()
+        unfused(uevs[i])
+    torch.cuda.synchronize()
+    if int(st_sel.item()) != 0 or int(st_score.item()) != 0:
+        raise RuntimeError("unfused score/select: device status")
+    if not torch.equal(kv_idx, kv_fused):
+        raise RuntimeError("the fused and the separate score/select calls selected different blocks")
+    uper = np.array([[uevs[i][j].elapsed_time(uevs[i][j + 1]) for j in range(2)] for i in range(5)])
+    unfused_ms = {"score_ms": float(uper[:, 0].mean()), "select_ms": float(uper[:, 1].mean())}
 
     # end to end through the C ABI with host buffers: every step copies its Q, K, V from
     # pinned host memory to the device and its O back, all inside the timed region. The
@@ -446,7 +474,7 @@ def main_gpu(args):
         score_kinds[kind] = {"ms": statistics.mean(a.elapsed_time(b_) for a, b_ in ts),
                              "beta": beta if kind == "vlog" else None}
         del kws
-    score_kinds["mean"] = {"ms": score_ms}
+    score_kinds["mean"] = {"ms": unfused_ms["score_ms"]}
 
     # vertical-slash attention on the 32k vertical-slash workload (timed on its own)
     vspec = S.WORKLOADS["prefill_32k_vs"]
@@ -586,8 +614,8 @@ def main_gpu(args):
                        "attend_tflop_per_step": flops / 1e12,
                        "l2": "256 MB buffer written between timed steps; inputs 1.6 GB > 126 MB L2",
                        "parallelism": f"independent problem per rank x{world}"},
-            "kernel_ms": {"score": score_ms, "select": select_ms, "attend": attend_ms},
-            "path_rooflines": path_rooflines(spec, score_ms, select_ms, peaks),
+            "kernel_ms": {"score_select": score_select_ms, "attend": attend_ms},
+            "path_rooflines": path_rooflines(spec, score_select_ms, unfused_ms, peaks),
             "score_backbones_ms": score_kinds,
             "vertical_slash": vs_res,
             "attend_detail": {"frac_of_burst_peak": achieved / burst, "burst_peak": burst,
@@ -596,7 +624,7 @@ def main_gpu(args):
                               "unmasked_pair_tflops": achieved_unmasked,
                               "unmasked_pairs": unmasked_pairs,
                               "step_ms_median": float(np.median(per.sum(axis=1))),
-                              "attend_ms_median": float(np.median(per[:, 2])),
+                              "attend_ms_median": float(np.median(per[:, 1])),
                               "warm_no_flush": warm},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst,
                          "unit": "TFLOP/s", "frac": achieved / burst, "traffic": traffic,
@@ -640,36 +668,45 @@ def unmasked_pair_count(torch, kv_idx, kv_cnt, tile_q, block_k):
     return float(((ramp + flat) * valid).sum().item())
 
 
-def path_rooflines(spec, score_ms, select_ms, peaks):
-    """Score and selection against their rooflines, from the workload's shape.
+def path_rooflines(spec, score_select_ms, unfused_ms, peaks):
+    """Scoring and selection against their rooflines, from the workload's shape.
 
-    Score (pool + score launches): 2 * d * tile_q flops per (b, h, tile, causal block j <= J_t),
-    the algorithmic count (the bf16 hi/lo split executes twice that), against the sustained
-    tensor peak; and its compulsory bytes (Q and K read, the causal scores written) against HBM.
-    Selection (rank + gate + finalize): the candidate scores j < f_lo(t) read and kv_idx
-    written, against HBM."""
+    Scores: 2 * d * tile_q flops per (b, h, tile, causal block j <= J_t), the algorithmic count.
+    The fused call (pool + score with in-kernel ranking + gate + finalize) must read Q and K and
+    write kv_idx and kv_cnt; nothing else has to reach DRAM. It is reported against the burst
+    tensor peak (flops) and against HBM (those bytes). The separate calls add the scores' round
+    trip: bsa_score writes the causal scores, bsa_select reads the candidates back and writes
+    kv_idx."""
     n_qt = spec.N // spec.tile_q
     causal = sum(((t + 1) * spec.tile_q - 1) // spec.block_k + 1 for t in range(n_qt))
     cand = sum((t * spec.tile_q) // spec.block_k for t in range(n_qt))
     heads = spec.B * spec.Hq
     W = min(spec.rho * max(spec.k_first, spec.k_last), spec.N // spec.block_k)
     score_flop = 2.0 * spec.d * spec.tile_q * causal * heads
-    score_bytes = (heads * spec.N * spec.d * 2 + spec.B * spec.Hkv * spec.N * spec.d * 2
-                   + heads * causal * 4)
+    qk_bytes = heads * spec.N * spec.d * 2 + spec.B * spec.Hkv * spec.N * spec.d * 2
+    kv_bytes = heads * n_qt * (W + 1) * 4
+    fused_bytes = qk_bytes + kv_bytes
+    score_bytes = qk_bytes + heads * causal * 4
     sel_bytes = heads * cand * 4 + heads * n_qt * W * 4
-    sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    sc_tflops = score_flop / (score_ms * 1e-3) / 1e12
-    sc_gbps = score_bytes / (score_ms * 1e-3) / 1e9
-    sel_gbps = sel_bytes / (select_ms * 1e-3) / 1e9
+    f_tflops = score_flop / (score_select_ms * 1e-3) / 1e12
+    f_gbps = fused_bytes / (score_select_ms * 1e-3) / 1e9
+    u_score, u_sel = unfused_ms["score_ms"], unfused_ms["select_ms"]
     return {
-        "score": {"ms": score_ms, "algorithmic_tflop": score_flop / 1e12, "tflops": sc_tflops,
-                  "frac_tensor_sustained": sc_tflops / sustained,
-                  "executed_frac_tensor_sustained": 2.0 * sc_tflops / sustained,
-                  "bytes": score_bytes, "GBps": sc_gbps, "frac_hbm": sc_gbps / hbm,
-                  "note": "pool + score launches; hi/lo split executes 2x the algorithmic flops"},
-        "select": {"ms": select_ms, "bytes": sel_bytes, "GBps": sel_gbps, "frac_hbm": sel_gbps / hbm,
-                   "note": "rank + gate + finalize; candidate scores read, kv_idx written"},
+        "score_select": {"ms": score_select_ms, "algorithmic_tflop": score_flop / 1e12,
+                         "tflops": f_tflops, "frac_tensor_burst": f_tflops / burst,
+                         "bytes": fused_bytes, "GBps": f_gbps, "frac_hbm": f_gbps / hbm,
+                         "note": "one bsa_score_select call: pool, score with the ranking in the "
+                                 "same kernel (fp16 operands, one pass), gate, finalize; Q and K "
+                                 "read, kv_idx and kv_cnt written"},
+        "unfused": {"score_ms": u_score, "select_ms": u_sel,
+                    "score_tflops": score_flop / (u_score * 1e-3) / 1e12,
+                    "score_GBps": score_bytes / (u_score * 1e-3) / 1e9,
+                    "select_GBps": sel_bytes / (u_sel * 1e-3) / 1e9,
+                    "select_frac_hbm": sel_bytes / (u_sel * 1e-3) / 1e9 / hbm,
+                    "note": "bsa_score (scores written) then bsa_select (candidate scores read back, "
+                            "kv_idx written), same inputs and selection"},
     }
 
 

@@ -33,7 +33,8 @@ EXPORTS = ("bsa_score_workspace_bytes", "bsa_score", "bsa_kv_idx_width",
            "bsa_select_workspace_bytes", "bsa_select", "bsa_attend", "bsa_decode",
            "bsa_status_string", "bsa_last_error", "bsa_select_noalloc_max_bytes",
            "bsa_select_noalloc", "bsa_selftest_wait", "bsa_decode_list", "bsa_score_ex",
-           "bsa_attend_vs_workspace_bytes", "bsa_attend_vs")
+           "bsa_attend_vs_workspace_bytes", "bsa_attend_vs", "bsa_score_select_workspace_bytes",
+           "bsa_score_select")
 
 
 class BsaError(RuntimeError):
@@ -103,6 +104,11 @@ def lib() -> ctypes.CDLL:
         L.bsa_decode_list.argtypes = [dsp, dpp, vp, vp, vp, i32p, i32p, ctypes.c_int, ctypes.c_float,
                                       vp, i32p, vp, i32p, vp]
         L.bsa_decode_list.restype = ctypes.c_int
+        L.bsa_score_select_workspace_bytes.argtypes = [sp, ctypes.c_int, pp]
+        L.bsa_score_select_workspace_bytes.restype = sz
+        L.bsa_score_select.argtypes = [sp, ctypes.c_int, ctypes.POINTER(ScoreParams), pp, vp, vp, vp, vp,
+                                       i32p, i32p, vp, vp, vp, vp, i32p, vp, sz, vp]
+        L.bsa_score_select.restype = ctypes.c_int
         L.bsa_select_noalloc_max_bytes.argtypes = []
         L.bsa_select_noalloc_max_bytes.restype = sz
         L.bsa_select_noalloc.argtypes = [sp, pp, vp, i32p, i32p, vp, vp, vp, vp, i32p, vp]
@@ -201,6 +207,20 @@ def bsa_select(shape, params, scores, kv_idx, kv_cnt, sigma, sigma_bar, trigger,
     _check(lib().bsa_select(ctypes.byref(shape), ctypes.byref(params), _ptr(scores), _ptr(kv_idx),
                             _ptr(kv_cnt), _ptr(sigma), _ptr(sigma_bar), _ptr(trigger), _ptr(theta),
                             _ptr(dev_status), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def bsa_score_select_workspace_bytes(shape: Shape, kind: int, params: SelectParams) -> int:
+    return lib().bsa_score_select_workspace_bytes(ctypes.byref(shape), kind, ctypes.byref(params))
+
+
+def bsa_score_select(shape, kind, score_params, params, q, k, v, scores, kv_idx, kv_cnt, sigma,
+                     sigma_bar, trigger, theta, dev_status, ws, ws_bytes, stream=None) -> None:
+    _check(lib().bsa_score_select(ctypes.byref(shape), kind,
+                                  ctypes.byref(score_params) if score_params is not None else None,
+                                  ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(scores),
+                                  _ptr(kv_idx), _ptr(kv_cnt), _ptr(sigma), _ptr(sigma_bar),
+                                  _ptr(trigger), _ptr(theta), _ptr(dev_status), _ptr(ws), ws_bytes,
+                                  _stream(stream)))
 
 
 def bsa_select_noalloc(shape, params, scores, kv_idx, kv_cnt, sigma, sigma_bar, trigger, theta,
@@ -351,16 +371,60 @@ def decode(q, k_cache, v_cache, *, block_kv: int, tau: float, phi: float, patien
     return out, used, trace, st
 
 
-def prefill(q, k, v, *, block_k: int, tile_q: int, cfg: SelectConfig, output_aware: bool = False,
-            scale: Optional[float] = None, stream=None, kind: Optional[str] = None, beta: float = 0.0):
-    """score -> select -> attend on the current stream; returns (out, selection dict, status)."""
+def score_select(q, k, v=None, *, block_k: int, tile_q: int, cfg: SelectConfig, kind: str = "mean",
+                 beta: float = 0.0, want_scores: bool = True, stream=None):
+    """Scores and selection in one call (bsa_score_select). Returns the selection dict of
+    ``select`` plus "scores" (None unless want_scores)."""
     shape = make_shape(q, k, block_k, tile_q)
-    st_score = torch.zeros(1, dtype=torch.int32, device=q.device)
-    s = score(q, k, v, block_k=block_k, tile_q=tile_q, output_aware=output_aware, stream=stream,
-              status=st_score, kind=kind, beta=beta)
-    sel = select(s, shape=shape, cfg=cfg, stream=stream)
-    sel["score_status"] = st_score
+    code = SCORE_KINDS[kind]
+    p = cfg.c()
+    dev = q.device
+    W = bsa_kv_idx_width(shape, p)
+    if W < 0:
+        raise BsaError(BSA_ERR_INVALID_ARG, lib().bsa_last_error().decode())
+    B, Hq, N, _ = q.shape
+    n_qt, n_kb = N // tile_q, N // block_k
+    r = dict(
+        kv_idx=torch.empty(B, Hq, n_qt, W, dtype=torch.int32, device=dev),
+        kv_cnt=torch.empty(B, Hq, n_qt, dtype=torch.int32, device=dev),
+        sigma=torch.empty(B, Hq, n_qt, dtype=torch.float32, device=dev),
+        sigma_bar=torch.empty(B, n_qt, dtype=torch.float32, device=dev),
+        trigger=torch.empty(B, n_qt, dtype=torch.uint8, device=dev),
+        theta=torch.empty(1, dtype=torch.float32, device=dev),
+        dev_status=torch.zeros(1, dtype=torch.int32, device=dev),
+        scores=(torch.empty(B, Hq, n_qt, n_kb, dtype=torch.float32, device=dev) if want_scores else None),
+        W=W)
+    nb = bsa_score_select_workspace_bytes(shape, code, p)
+    if nb == 0:
+        raise BsaError(BSA_ERR_INVALID_ARG, lib().bsa_last_error().decode())
+    ws = _empty_bytes(nb, dev)
+    uses_v = kind in ("vnorm", "vlog")
+    bsa_score_select(shape, code, ScoreParams(beta), p, q, k, v if uses_v else None, r["scores"],
+                     r["kv_idx"], r["kv_cnt"], r["sigma"], r["sigma_bar"], r["trigger"], r["theta"],
+                     r["dev_status"], ws, nb, stream)
+    return r
+
+
+def prefill(q, k, v, *, block_k: int, tile_q: int, cfg: SelectConfig, output_aware: bool = False,
+            scale: Optional[float] = None, stream=None, kind: Optional[str] = None, beta: float = 0.0,
+            fused: bool = True):
+    """score -> select -> attend on the current stream; returns (out, selection dict, status).
+    fused: scores and selection in one bsa_score_select call (scores written out too);
+    otherwise bsa_score then bsa_select."""
+    shape = make_shape(q, k, block_k, tile_q)
+    if kind is None:
+        kind = "vnorm" if output_aware else "mean"
+    if fused:
+        sel = score_select(q, k, v, block_k=block_k, tile_q=tile_q, cfg=cfg, kind=kind, beta=beta,
+                           want_scores=True, stream=stream)
+        sel["score_status"] = torch.zeros(1, dtype=torch.int32, device=q.device)
+    else:
+        st_score = torch.zeros(1, dtype=torch.int32, device=q.device)
+        s = score(q, k, v, block_k=block_k, tile_q=tile_q, stream=stream, status=st_score, kind=kind,
+                  beta=beta)
+        sel = select(s, shape=shape, cfg=cfg, stream=stream)
+        sel["score_status"] = st_score
+        sel["scores"] = s
     out, _, st = attend(q, k, v, sel["kv_idx"], sel["kv_cnt"], block_k=block_k, tile_q=tile_q,
                         scale=scale, stream=stream)
-    sel["scores"] = s
     return out, sel, st

@@ -66,9 +66,11 @@ bsa_status check_params(const bsa_shape* s, const bsa_select_params* p) {
 struct ScoreWs {
   float* kbar;       // pooled keys, or kmin (bounds)
   float* kbar2;      // kmax (bounds)
-  uint16_t* hi;      // bf16 split of kbar, or of mid (bounds)
+  uint16_t* h16;     // fp16 pooled keys scaled by 2^r per block (mean kinds, tensor cores)
+  float* kinv;       // 2^-r per block
+  uint16_t* hi;      // bounds, tensor cores: bf16 hi/lo of mid and rad
   uint16_t* lo;
-  uint16_t* hi2;     // bf16 split of rad (bounds)
+  uint16_t* hi2;
   uint16_t* lo2;
   float* w;          // value-block term (output-aware kinds)
   size_t bytes;
@@ -87,12 +89,15 @@ ScoreWs score_ws(const bsa_shape& s, bsa_score_kind kind, void* base) {
   size_t off = 0;
   char* p = (char*)base;
   w.kbar = (float*)(p + off); off += align256(nk * s.d * 4);
-  w.hi = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
-  w.lo = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
   if (bounds) {
     w.kbar2 = (float*)(p + off); off += align256(nk * s.d * 4);
+    w.hi = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
+    w.lo = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
     w.hi2 = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
     w.lo2 = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
+  } else {
+    w.h16 = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
+    w.kinv = (float*)(p + off); off += align256(nk * 4);
   }
   if (vterm) {
     w.w = (float*)(p + off); off += align256(nk * 4);
@@ -153,47 +158,128 @@ size_t bsa_score_workspace_bytes(const bsa_shape* s, bsa_score_kind kind) {
   return score_ws(*s, kind, nullptr).bytes;
 }
 
-bsa_status bsa_score_ex(const bsa_shape* s, bsa_score_kind kind, const bsa_score_params* prm,
-                        const void* q, const void* k, const void* v, float* scores,
-                        int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Argument checks shared by bsa_score_ex and bsa_score_select; returns beta in *beta.
+bsa_status check_score_args(const bsa_shape* s, bsa_score_kind kind, const bsa_score_params* prm,
+                            const void* q, const void* k, const void* v, float* beta) {
   bsa_status st = check_shape(s);
   if (st != BSA_OK) return st;
   if (!known_kind(kind)) return fail(BSA_ERR_INVALID_ARG, "unknown score kind");
-  if (!q || !k || !scores || !ws) return fail(BSA_ERR_INVALID_ARG, "NULL q, k, scores or workspace");
+  if (!q || !k) return fail(BSA_ERR_INVALID_ARG, "NULL q or k");
   const bool vterm = kind == BSA_SCORE_MEAN_VNORM || kind == BSA_SCORE_MEAN_VLOG;
   if (vterm && !v) return fail(BSA_ERR_INVALID_ARG, "v is NULL for an output-aware score");
-  float beta = 0.f;
+  *beta = 0.f;
   if (kind == BSA_SCORE_MEAN_VLOG) {
     if (!prm) return fail(BSA_ERR_INVALID_ARG, "BSA_SCORE_MEAN_VLOG needs params (beta)");
-    beta = prm->beta;
-    if (!(beta >= 0.f) || !(beta < INFINITY)) return fail(BSA_ERR_INVALID_ARG, "beta must be finite and >= 0");
+    *beta = prm->beta;
+    if (!(*beta >= 0.f) || !(*beta < INFINITY)) return fail(BSA_ERR_INVALID_ARG, "beta must be finite and >= 0");
   }
-  if (!aligned16(q) || !aligned16(k) || (v && !aligned16(v)) || ((uintptr_t)ws & 255u))
-    return fail(BSA_ERR_INVALID_ARG, "q/k/v need 16-byte and workspace 256-byte alignment");
+  if (!aligned16(q) || !aligned16(k) || (v && !aligned16(v)))
+    return fail(BSA_ERR_INVALID_ARG, "q/k/v need 16-byte alignment");
+  return BSA_OK;
+}
+
+int wmode_of(bsa_score_kind kind) {
+  return kind == BSA_SCORE_MEAN_VNORM ? 1 : (kind == BSA_SCORE_MEAN_VLOG ? 2 : 0);
+}
+
+// Pool (+ value term) and, unless ranked is given with the fused kernel, the scores.
+// Launches only; the arguments are checked.
+bsa_status run_score(const bsa_shape& s, bsa_score_kind kind, float beta, const void* q, const void* k,
+                     const void* v, float* scores, int32_t* dev_status, const ScoreWs& w, cudaStream_t cs) {
+  cudaError_t e;
+  if (kind == BSA_SCORE_KMINMAX) {
+    const bool tc = bsa::score_tc_supported(s);
+    e = bsa::launch_pool_bounds(s, k, w.kbar, w.kbar2, tc ? w.hi : nullptr, w.lo, w.hi2, w.lo2, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "pool (bounds)");
+    e = tc ? bsa::launch_score_tc_bounds(s, q, w.hi, w.lo, w.hi2, w.lo2, scores, dev_status, cs)
+           : bsa::launch_score_simt(s, q, w.kbar, w.kbar2, nullptr, 0, scores, cs);
+    if (e != cudaSuccess) return cuda_fail(e, tc ? "score (tensor cores)" : "score");
+    return BSA_OK;
+  }
+  const bool vterm = kind == BSA_SCORE_MEAN_VNORM || kind == BSA_SCORE_MEAN_VLOG;
+  const bool tc = bsa::score_rank_supported(s);
+  e = bsa::launch_pool(s, k, vterm ? v : nullptr, w.kbar, tc ? w.h16 : nullptr, w.kinv, w.w, cs,
+                       kind == BSA_SCORE_MEAN_VLOG ? 1 : 0, beta);
+  if (e != cudaSuccess) return cuda_fail(e, "pool");
+  e = tc ? bsa::launch_score_rank(s, nullptr, q, w.h16, w.kinv, w.w, wmode_of(kind), scores, nullptr, 0,
+                                  nullptr, nullptr, 0, dev_status, cs)
+         : bsa::launch_score_simt(s, q, w.kbar, nullptr, w.w, wmode_of(kind), scores, cs);
+  if (e != cudaSuccess) return cuda_fail(e, tc ? "score (tensor cores)" : "score");
+  return BSA_OK;
+}
+
+// Gate and kv_idx from the ranked lists and sigma.
+bsa_status run_gate_finalize(const bsa_shape& s, const bsa_select_params& p, int W, const SelectWs& w,
+                             const float* sg, float* sigma_bar, uint8_t* trigger, float* theta,
+                             int32_t* kv_idx, int32_t* kv_cnt, cudaStream_t cs) {
+  float* sb = sigma_bar ? sigma_bar : w.sigma_bar;
+  uint8_t* tr = trigger ? trigger : w.trigger;
+  cudaError_t e = bsa::launch_gate(s, p, sg, sb, tr, theta, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "gate");
+  e = bsa::launch_finalize(s, p, w.ranked, W, tr, W, kv_idx, kv_cnt, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "finalize");
+  return BSA_OK;
+}
+
+// Workspace of bsa_score_select: the score workspace, the selection workspace, and either
+// the row ring of the fused kernel or (for the shapes and kinds it does not take) a scores
+// array for the unfused path.
+struct ScoreSelectWs {
+  ScoreWs sc;
+  SelectWs sel;
+  float* ring;       // fused: [kScoreRankRingCtas][2][heads per unit][n_kb]
+  float* scores;     // unfused: [B,Hq,n_qt,n_kb]
+  size_t bytes;
+};
+
+bool fused_kind(bsa_score_kind kind) {
+  return kind == BSA_SCORE_MEAN || kind == BSA_SCORE_MEAN_VNORM || kind == BSA_SCORE_MEAN_VLOG;
+}
+
+ScoreSelectWs score_select_ws(const bsa_shape& s, bsa_score_kind kind, int W, void* base) {
+  ScoreSelectWs w{};
+  char* p = (char*)base;
+  w.sc = score_ws(s, kind, p);
+  size_t off = w.sc.bytes;
+  w.sel = select_ws(s, W, p ? p + off : nullptr);
+  off += w.sel.bytes;
+  const size_t n_kb = (size_t)(s.N / s.block_k);
+  if (fused_kind(kind) && bsa::score_rank_supported(s)) {
+    w.ring = (float*)(p + off);
+    off += align256((size_t)bsa::kScoreRankRingCtas * 2 * bsa::score_rank_heads_per_unit(s) * n_kb * 4);
+  } else {
+    w.scores = (float*)(p + off);
+    off += align256((size_t)s.B * s.Hq * (s.N / s.tile_q) * n_kb * 4);
+  }
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+bsa_status bsa_score_ex(const bsa_shape* s, bsa_score_kind kind, const bsa_score_params* prm,
+                        const void* q, const void* k, const void* v, float* scores,
+                        int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  float beta;
+  bsa_status st = check_score_args(s, kind, prm, q, k, v, &beta);
+  if (st != BSA_OK) return st;
+  if (!scores || !ws) return fail(BSA_ERR_INVALID_ARG, "NULL scores or workspace");
+  if ((uintptr_t)ws & 255u) return fail(BSA_ERR_INVALID_ARG, "workspace needs 256-byte alignment");
   ScoreWs w = score_ws(*s, kind, ws);
   if (ws_bytes < w.bytes) return fail(BSA_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, w.bytes);
   cudaStream_t cs = (cudaStream_t)stream;
-  cudaError_t e;
   if (dev_status) {
-    e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
+    cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
     if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
   }
-  const bool tc = bsa::score_tc_supported(*s);      // tensor cores for bf16, d 128, tiles of 128
-  const int wmode = kind == BSA_SCORE_MEAN_VNORM ? 1 : (kind == BSA_SCORE_MEAN_VLOG ? 2 : 0);
-  if (kind == BSA_SCORE_KMINMAX) {
-    e = bsa::launch_pool_bounds(*s, k, w.kbar, w.kbar2, tc ? w.hi : nullptr, w.lo, w.hi2, w.lo2, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "pool (bounds)");
-    e = tc ? bsa::launch_score_tc(*s, q, w.hi, w.lo, nullptr, 0, scores, dev_status, cs, w.hi2, w.lo2)
-           : bsa::launch_score_simt(*s, q, w.kbar, w.kbar2, nullptr, 0, scores, cs);
-  } else {
-    e = bsa::launch_pool(*s, k, vterm ? v : nullptr, w.kbar, tc ? w.hi : nullptr, w.lo, w.w, cs,
-                         kind == BSA_SCORE_MEAN_VLOG ? 1 : 0, beta);
-    if (e != cudaSuccess) return cuda_fail(e, "pool");
-    e = tc ? bsa::launch_score_tc(*s, q, w.hi, w.lo, w.w, wmode, scores, dev_status, cs)
-           : bsa::launch_score_simt(*s, q, w.kbar, nullptr, w.w, wmode, scores, cs);
-  }
-  if (e != cudaSuccess) return cuda_fail(e, tc ? "score (tensor cores)" : "score");
-  return ok();
+  st = run_score(*s, kind, beta, q, k, v, scores, dev_status, w, cs);
+  return st == BSA_OK ? ok() : st;
 }
 
 bsa_status bsa_score(const bsa_shape* s, bsa_score_kind kind, const void* q, const void* k,
@@ -236,15 +322,59 @@ bsa_status bsa_select(const bsa_shape* s, const bsa_select_params* p, const floa
     if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
   }
   float* sg = sigma ? sigma : w.sigma;
-  float* sb = sigma_bar ? sigma_bar : w.sigma_bar;
-  uint8_t* tr = trigger ? trigger : w.trigger;
   e = bsa::launch_select_rank(*s, *p, scores, W, w.ranked, sg, dev_status, cs);
   if (e != cudaSuccess) return cuda_fail(e, "select_rank");
-  e = bsa::launch_gate(*s, *p, sg, sb, tr, theta, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "gate");
-  e = bsa::launch_finalize(*s, *p, w.ranked, W, tr, W, kv_idx, kv_cnt, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "finalize");
-  return ok();
+  st = run_gate_finalize(*s, *p, W, w, sg, sigma_bar, trigger, theta, kv_idx, kv_cnt, cs);
+  return st == BSA_OK ? ok() : st;
+}
+
+size_t bsa_score_select_workspace_bytes(const bsa_shape* s, bsa_score_kind kind,
+                                        const bsa_select_params* p) {
+  if (check_shape(s) != BSA_OK || !known_kind(kind) || check_params(s, p) != BSA_OK) return 0;
+  const int W = bsa::kv_width(s->N, s->tile_q, s->block_k, p->k_first, p->k_last, p->rho);
+  return score_select_ws(*s, kind, W, nullptr).bytes;
+}
+
+bsa_status bsa_score_select(const bsa_shape* s, bsa_score_kind kind, const bsa_score_params* prm,
+                            const bsa_select_params* p, const void* q, const void* k, const void* v,
+                            float* scores, int32_t* kv_idx, int32_t* kv_cnt, float* sigma,
+                            float* sigma_bar, uint8_t* trigger, float* theta, int32_t* dev_status,
+                            void* ws, size_t ws_bytes, void* stream) {
+  float beta;
+  bsa_status st = check_score_args(s, kind, prm, q, k, v, &beta);
+  if (st != BSA_OK) return st;
+  st = check_params(s, p);
+  if (st != BSA_OK) return st;
+  if (!kv_idx || !kv_cnt || !ws) return fail(BSA_ERR_INVALID_ARG, "NULL kv_idx, kv_cnt or workspace");
+  if ((uintptr_t)ws & 255u) return fail(BSA_ERR_INVALID_ARG, "workspace needs 256-byte alignment");
+  const int W = bsa::kv_width(s->N, s->tile_q, s->block_k, p->k_first, p->k_last, p->rho);
+  ScoreSelectWs w = score_select_ws(*s, kind, W, ws);
+  if (ws_bytes < w.bytes) return fail(BSA_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, w.bytes);
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e;
+  if (dev_status) {
+    e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
+  }
+  float* sg = sigma ? sigma : w.sel.sigma;
+  if (w.ring) {
+    // fused: scores are ranked inside the score kernel and written only when asked for
+    const bool vterm = kind == BSA_SCORE_MEAN_VNORM || kind == BSA_SCORE_MEAN_VLOG;
+    e = bsa::launch_pool(*s, k, vterm ? v : nullptr, w.sc.kbar, w.sc.h16, w.sc.kinv, w.sc.w, cs,
+                         kind == BSA_SCORE_MEAN_VLOG ? 1 : 0, beta);
+    if (e != cudaSuccess) return cuda_fail(e, "pool");
+    e = bsa::launch_score_rank(*s, p, q, w.sc.h16, w.sc.kinv, w.sc.w, wmode_of(kind), scores, w.ring,
+                               bsa::kScoreRankRingCtas, w.sel.ranked, sg, W, dev_status, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "score+rank (tensor cores)");
+  } else {
+    float* sc = scores ? scores : w.scores;
+    st = run_score(*s, kind, beta, q, k, v, sc, dev_status, w.sc, cs);
+    if (st != BSA_OK) return st;
+    e = bsa::launch_select_rank(*s, *p, sc, W, w.sel.ranked, sg, dev_status, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "select_rank");
+  }
+  st = run_gate_finalize(*s, *p, W, w.sel, sg, sigma_bar, trigger, theta, kv_idx, kv_cnt, cs);
+  return st == BSA_OK ? ok() : st;
 }
 
 bsa_status bsa_attend(const bsa_shape* s, const void* q, const void* k, const void* v,

@@ -8,11 +8,12 @@
 
 namespace bsa {
 
-// Pooled keys (+ value-block term). kbar fp32 [B,Hkv,n_kb,d]; kbar_hi/lo bf16 split of
-// kbar (may be null); wnorm [B,Hkv,n_kb] (only when v != null): ||Vbar|| (wlog 0) or
-// beta * max(0, ln ||Vbar||^2) (wlog 1).
+// Pooled keys (+ value-block term). kbar fp32 [B,Hkv,n_kb,d]; kbar16 fp16 [B,Hkv,n_kb,d]
+// scaled per block by 2^r and kinv [B,Hkv,n_kb] = 2^-r (both may be null); wnorm
+// [B,Hkv,n_kb] (only when v != null): ||Vbar|| (wlog 0) or beta * max(0, ln ||Vbar||^2)
+// (wlog 1).
 cudaError_t launch_pool(const bsa_shape& s, const void* k, const void* v, float* kbar,
-                        uint16_t* kbar_hi, uint16_t* kbar_lo, float* wnorm, cudaStream_t st,
+                        uint16_t* kbar16, float* kinv, float* wnorm, cudaStream_t st,
                         int wlog = 0, float beta = 0.f);
 
 // Per-coordinate key bounds: kmin, kmax fp32 [B,Hkv,n_kb,d]; for the tensor-core score
@@ -27,13 +28,26 @@ cudaError_t launch_score_simt(const bsa_shape& s, const void* q, const float* kb
                               const float* kbar2, const float* wnorm, int wmode, float* scores,
                               cudaStream_t st);
 
-// Block scores on tcgen05 tensor cores (bf16 inputs, hi/lo split of the pooled keys;
-// with rad_hi/lo given, the bounds backbone with kbar_hi/lo = mid).
+// K-min/K-max block scores on tcgen05 tensor cores (bf16 inputs; mid and rad of the key
+// boxes as bf16 hi/lo pairs).
 bool score_tc_supported(const bsa_shape& s);
-cudaError_t launch_score_tc(const bsa_shape& s, const void* q, const uint16_t* kbar_hi,
-                            const uint16_t* kbar_lo, const float* wnorm, int wmode, float* scores,
-                            int32_t* dev_status, cudaStream_t st, const uint16_t* rad_hi = nullptr,
-                            const uint16_t* rad_lo = nullptr);
+cudaError_t launch_score_tc_bounds(const bsa_shape& s, const void* q, const uint16_t* mid_hi,
+                                   const uint16_t* mid_lo, const uint16_t* rad_hi,
+                                   const uint16_t* rad_lo, float* scores, int32_t* dev_status,
+                                   cudaStream_t st);
+
+// Mean-pooled block scores on tcgen05 (fp16 operands with power-of-two scales), persistent,
+// optionally fused with the ranking of the selection. kbar16/kinv from launch_pool.
+// ranked == null: scores only (scores required). ranked != null: also the top-M lists
+// [B*Hq*n_qt][W] and sigma; scores may then be null, and the rows go through
+// ring [ring_ctas][2][heads per unit][n_kb] instead (the grid is capped at ring_ctas).
+bool score_rank_supported(const bsa_shape& s);
+int score_rank_heads_per_unit(const bsa_shape& s);
+constexpr int kScoreRankRingCtas = 256;
+cudaError_t launch_score_rank(const bsa_shape& s, const bsa_select_params* p, const void* q,
+                              const uint16_t* kbar16, const float* kinv, const float* wnorm, int wmode,
+                              float* scores, float* ring, int ring_ctas, int32_t* ranked, float* sigma,
+                              int W, int32_t* dev_status, cudaStream_t st);
 
 // Selection: ranked candidate lists + sigma, then the gate, then kv_idx.
 cudaError_t launch_select_rank(const bsa_shape& s, const bsa_select_params& p, const float* scores,

@@ -13,6 +13,8 @@
 // (times w_j, or plus w_j, for the output-aware forms), or of
 // sum_c max(q_ic kmin_jc, q_ic kmax_jc) for the bounds backbone; -inf for
 // blocks the tile cannot see.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -20,17 +22,22 @@ namespace bsa {
 
 // One CTA per (b, g, key block). 256 threads: each thread owns 8 consecutive
 // columns (one 16-byte load for bf16) and a phase of the rows.
+// With kbar16 given, the pooled keys are also written as fp16 scaled by a power of two
+// 2^r per block (r chosen so that the block's largest |Kbar| lands in [2^14, 2^15)), with
+// kinv[block] = 2^-r: the operand of the tensor-core score.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ k, const T* __restrict__ v,
                                                    int N, int block_k, float* __restrict__ kbar,
-                                                   uint16_t* __restrict__ kbar_hi,
-                                                   uint16_t* __restrict__ kbar_lo,
+                                                   uint16_t* __restrict__ kbar16,
+                                                   float* __restrict__ kinv,
                                                    float* __restrict__ wnorm, int wlog, float beta) {
   constexpr int CPT = 8;                 // columns per thread
   constexpr int TPR = D / CPT;           // threads per row
   constexpr int PHASES = 256 / TPR;      // rows in flight
   __shared__ float red[PHASES][D];
   __shared__ float vsum[D];
+  __shared__ float mrow[D];
+  __shared__ int rexp;
   const int j = blockIdx.x;
   const size_t bg = blockIdx.y;
   const int n_kb = N / block_k;
@@ -65,18 +72,37 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ k, cons
       for (int p = 0; p < PHASES; ++p) s += red[p][c];
       float mean = s * inv;
       if (pass == 0) {
-        size_t o = (bg * n_kb + j) * D + c;
-        kbar[o] = mean;
-        if (kbar_hi) {
-          uint16_t hi = f32_to_bf16_rn(mean);
-          kbar_hi[o] = hi;
-          kbar_lo[o] = f32_to_bf16_rn(mean - bf16_to_f32(hi));
-        }
+        kbar[(bg * n_kb + j) * D + c] = mean;
+        mrow[c] = mean;
       } else {
         vsum[c] = mean * mean;
       }
     }
     __syncthreads();
+    if (pass == 0 && kbar16) {
+      if (threadIdx.x < 32) {
+        float mx = 0.f;
+        for (int c = threadIdx.x; c < D; c += 32) mx = fmaxf(mx, fabsf(mrow[c]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (threadIdx.x == 0) {
+          const uint32_t u = __float_as_uint(mx);
+          int r = 0;
+          if (u != 0u && u < 0x7f800000u) {
+            r = 14 - ((int)(u >> 23) - 127);
+            r = r < -126 ? -126 : (r > 126 ? 126 : r);
+          }
+          rexp = r;
+          kinv[bg * n_kb + j] = __int_as_float((127 - r) << 23);
+        }
+      }
+      __syncthreads();
+      const float sc = __int_as_float((127 + rexp) << 23);
+      for (int c = threadIdx.x; c < D; c += blockDim.x) {
+        const __half h = __float2half_rn(mrow[c] * sc);
+        kbar16[(bg * n_kb + j) * D + c] = *reinterpret_cast<const uint16_t*>(&h);
+      }
+    }
   }
   if (v && threadIdx.x < 32) {
     float s = 0.f;
@@ -142,26 +168,26 @@ __global__ void __launch_bounds__(256) pool_bounds_kernel(const T* __restrict__ 
 }
 
 cudaError_t launch_pool(const bsa_shape& s, const void* k, const void* v, float* kbar,
-                        uint16_t* kbar_hi, uint16_t* kbar_lo, float* wnorm, cudaStream_t st,
+                        uint16_t* kbar16, float* kinv, float* wnorm, cudaStream_t st,
                         int wlog, float beta) {
   dim3 grid(s.N / s.block_k, s.B * s.Hkv);
   if (s.dtype == BSA_BF16) {
     auto kk = (const uint16_t*)k;
     auto vv = (const uint16_t*)v;
     if (s.d == 128)
-      pool_kernel<uint16_t, 128><<<grid, 256, 0, st>>>(kk, vv, s.N, s.block_k, kbar, kbar_hi, kbar_lo, wnorm,
+      pool_kernel<uint16_t, 128><<<grid, 256, 0, st>>>(kk, vv, s.N, s.block_k, kbar, kbar16, kinv, wnorm,
                                                        wlog, beta);
     else
-      pool_kernel<uint16_t, 64><<<grid, 256, 0, st>>>(kk, vv, s.N, s.block_k, kbar, kbar_hi, kbar_lo, wnorm,
+      pool_kernel<uint16_t, 64><<<grid, 256, 0, st>>>(kk, vv, s.N, s.block_k, kbar, kbar16, kinv, wnorm,
                                                       wlog, beta);
   } else {
     auto kk = (const float*)k;
     auto vv = (const float*)v;
     if (s.d == 128)
-      pool_kernel<float, 128><<<grid, 256, 0, st>>>(kk, vv, s.N, s.block_k, kbar, kbar_hi, kbar_lo, wnorm,
+      pool_kernel<float, 128><<<grid, 256, 0, st>>>(kk, vv, s.N, s.block_k, kbar, kbar16, kinv, wnorm,
                                                     wlog, beta);
     else
-      pool_kernel<float, 64><<<grid, 256, 0, st>>>(kk, vv, s.N, s.block_k, kbar, kbar_hi, kbar_lo, wnorm,
+      pool_kernel<float, 64><<<grid, 256, 0, st>>>(kk, vv, s.N, s.block_k, kbar, kbar16, kinv, wnorm,
                                                    wlog, beta);
   }
   return cudaGetLastError();

@@ -1,4 +1,6 @@
-// Block scores on Blackwell tensor cores (tcgen05 + TMEM + TMA).
+// K-min/K-max block scores on Blackwell tensor cores (tcgen05 + TMEM + TMA). The
+// mean-pooled backbones run in score_rank.cu; this kernel keeps the two-operand bounds
+// form with bf16 hi/lo operands.
 //
 // s(t,j) = max over the tile's rows i of q_i . Kbar_j ([UGS] step 2: the
 // tile's block score is the max over its rows; step 1: mean-pooled keys),
@@ -279,24 +281,18 @@ static cudaError_t launch_score_tc_t(const bsa_shape& s, const CUtensorMap& mq, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_score_tc(const bsa_shape& s, const void* q, const uint16_t* kbar_hi,
-                            const uint16_t* kbar_lo, const float* wnorm, int wmode, float* scores,
-                            int32_t* dev_status, cudaStream_t st, const uint16_t* rad_hi,
-                            const uint16_t* rad_lo) {
+cudaError_t launch_score_tc_bounds(const bsa_shape& s, const void* q, const uint16_t* mid_hi,
+                                   const uint16_t* mid_lo, const uint16_t* rad_hi,
+                                   const uint16_t* rad_lo, float* scores, int32_t* dev_status,
+                                   cudaStream_t st) {
   CUtensorMap mq, mh, ml, mh2, ml2;
   const uint64_t qrows = (uint64_t)s.B * s.Hq * s.N;
   const uint64_t krows = (uint64_t)s.B * s.Hkv * (s.N / s.block_k);
-  if (!make_tmap_bf16_2d(&mq, q, qrows, HD, 64, TQ) || !make_tmap_bf16_2d(&mh, kbar_hi, krows, HD, 64, CB) ||
-      !make_tmap_bf16_2d(&ml, kbar_lo, krows, HD, 64, CB))
+  if (!make_tmap_bf16_2d(&mq, q, qrows, HD, 64, TQ) || !make_tmap_bf16_2d(&mh, mid_hi, krows, HD, 64, CB) ||
+      !make_tmap_bf16_2d(&ml, mid_lo, krows, HD, 64, CB) || !make_tmap_bf16_2d(&mh2, rad_hi, krows, HD, 64, CB) ||
+      !make_tmap_bf16_2d(&ml2, rad_lo, krows, HD, 64, CB))
     return cudaErrorInvalidValue;
-  if (rad_hi) {
-    if (!make_tmap_bf16_2d(&mh2, rad_hi, krows, HD, 64, CB) || !make_tmap_bf16_2d(&ml2, rad_lo, krows, HD, 64, CB))
-      return cudaErrorInvalidValue;
-    return launch_score_tc_t<1, true>(s, mq, mh, ml, mh2, ml2, nullptr, 0, scores, dev_status, st);
-  }
-  const int G = s.Hq / s.Hkv;
-  if (G % 2 == 0) return launch_score_tc_t<2, false>(s, mq, mh, ml, mh, ml, wnorm, wmode, scores, dev_status, st);
-  return launch_score_tc_t<1, false>(s, mq, mh, ml, mh, ml, wnorm, wmode, scores, dev_status, st);
+  return launch_score_tc_t<1, true>(s, mq, mh, ml, mh2, ml2, nullptr, 0, scores, dev_status, st);
 }
 
 }  // namespace bsa

@@ -221,13 +221,20 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 
 // ---------------------------------------------------------------------------
-// tcgen05.mma, kind::f16 (bf16 x bf16 -> fp32), A and B from shared memory.
+// tcgen05.mma, kind::f16 (bf16 x bf16 or fp16 x fp16 -> fp32, by the instruction
+// descriptor; A and B always of one type), A and B from shared memory.
 
 // Instruction descriptor: fp32 accumulator (bits 4-5 = 1), A and B bf16 (bits 7-9 and
 // 10-12 = 1), A/B major (bits 15 / 16: 0 = K-major, 1 = MN-major), N>>3 at bits 17-22,
 // M>>4 at bits 24-28.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// The same with A and B fp16 (bits 7-9 and 10-12 = 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 

@@ -8,9 +8,12 @@ device), then optionally the decode path on a shortened cache.
 With --select-only the scores are computed once, Q, K and V are released, and
 only the selection runs (--iters times): at --n 131072 --heads 16 this is the
 full-length selection of half the heads (134 MB of scores, ~0.2 GB held).
+With --score-select only the scoring+selection call runs (--iters times), as the
+benchmark's step calls it (ranking inside the score kernel, no scores written).
 
     python -m block_sparse_causal_bsa_b200.profcase [--n 16384] [--heads 32] [--iters 2]
                                                     [--decode-len 8192] [--select-only]
+                                                    [--score-select]
 """
 from __future__ import annotations
 
@@ -36,6 +39,7 @@ def main():
     ap.add_argument("--decode-len", type=int, default=0)
     ap.add_argument("--heads", type=int, default=32)
     ap.add_argument("--select-only", action="store_true")
+    ap.add_argument("--score-select", action="store_true")
     a = ap.parse_args()
     spec = S.WORKLOADS["gated_prefill_128k"].scaled(N=a.n, Hq=a.heads, Hkv=max(1, a.heads // 4))
     q, k, v = S.prefill_inputs(spec, 7)
@@ -51,6 +55,16 @@ def main():
         torch.cuda.synchronize()
         status = int(sel["dev_status"].item())
         print(f"select N={a.n} Hq={a.heads}: selected blocks {int(sel['kv_cnt'].sum())}, status {status}")
+        if status:
+            raise SystemExit(f"device status {status}")
+        return
+    if a.score_select:
+        for _ in range(a.iters):
+            sel = bb.score_select(qd, kd, vd, block_k=spec.block_k, tile_q=spec.tile_q, cfg=cfg,
+                                  want_scores=False)
+        torch.cuda.synchronize()
+        status = int(sel["dev_status"].item())
+        print(f"score_select N={a.n} Hq={a.heads}: selected blocks {int(sel['kv_cnt'].sum())}, status {status}")
         if status:
             raise SystemExit(f"device status {status}")
         return

@@ -160,7 +160,14 @@ size_t bsa_score_workspace_bytes(const bsa_shape* shape, bsa_score_kind kind);
  * q, k: inputs of `shape->dtype`; v is read only for the output-aware kinds (VNORM, VLOG;
  * else may be NULL).
  * dev_status: device int32 or NULL (BSA_DEV_TIMEOUT if a bounded wait ran out).
- * bsa_score takes every kind but BSA_SCORE_MEAN_VLOG (which needs beta: INVALID_ARG). */
+ * bsa_score takes every kind but BSA_SCORE_MEAN_VLOG (which needs beta: INVALID_ARG).
+ * Precision: bf16 inputs with d = 128 and query tiles of 128 score the mean-pooled
+ * kinds on tensor cores with fp16 operands: each query tile and each pooled-key block
+ * is scaled by a power of two (exact) so that its largest magnitude lands in
+ * [2^14, 2^15); the pooled keys are then rounded to fp16 (relative 2^-12), the query
+ * values convert exactly unless they lie more than 2^-24 below the tile's largest, and
+ * the products accumulate in fp32. BSA_SCORE_KMINMAX on tensor cores carries the box
+ * centre and half-width as bf16 hi/lo pairs (about 2^-17 relative). */
 bsa_status bsa_score(const bsa_shape* shape, bsa_score_kind kind,
                      const void* q, const void* k, const void* v,
                      float* scores, int32_t* dev_status, void* workspace, size_t workspace_bytes,
@@ -200,6 +207,35 @@ bsa_status bsa_select(const bsa_shape* shape, const bsa_select_params* params,
                       float* sigma, float* sigma_bar, uint8_t* trigger, float* theta,
                       int32_t* dev_status, void* workspace, size_t workspace_bytes,
                       void* stream);
+
+/* ---- scoring and selection in one call ([UGS] steps 1-5; [Stem] 2.A, 2.B) -------- */
+
+/* Workspace bytes bsa_score_select needs (0 on invalid arguments). */
+size_t bsa_score_select_workspace_bytes(const bsa_shape* shape, bsa_score_kind kind,
+                                        const bsa_select_params* params);
+
+/* bsa_score followed by bsa_select, with the same arguments and results, in one call:
+ * the pages' framing of scores -> per-tile top-k -> kv_idx ([UGS] steps 2-5; its
+ * Contribuições 3 runs selection and expansion in one fused code path).
+ *   scores   [B,Hq,n_qt,n_kb] fp32 or NULL. NULL: the scores are not written out.
+ *   kv_idx, kv_cnt, sigma, sigma_bar, trigger, theta, dev_status: as bsa_select
+ *            (dev_status also collects bsa_score's device bits).
+ *   params   score parameters as bsa_score_ex (NULL except for BSA_SCORE_MEAN_VLOG).
+ * For bf16 inputs with d = 128 and query tiles of 128, and the mean-pooled kinds
+ * (BSA_SCORE_MEAN, _VNORM, _VLOG), the ranking runs inside the tensor-core score
+ * kernel: each (batch, head, tile) row is ranked by a warp of the score kernel
+ * right after it is complete, from L2, and the scores never make a round trip
+ * through DRAM unless asked for. Other shapes and BSA_SCORE_KMINMAX run the two
+ * calls one after the other (the scores then pass through the workspace when the
+ * scores pointer is NULL). Results are identical either way given the same scores.
+ * Workspace: bsa_score_select_workspace_bytes() bytes, 256-byte aligned. Errors,
+ * limits and stream semantics as bsa_score and bsa_select. */
+bsa_status bsa_score_select(const bsa_shape* shape, bsa_score_kind kind,
+                            const bsa_score_params* score_params, const bsa_select_params* params,
+                            const void* q, const void* k, const void* v, float* scores,
+                            int32_t* kv_idx, int32_t* kv_cnt, float* sigma, float* sigma_bar,
+                            uint8_t* trigger, float* theta, int32_t* dev_status, void* workspace,
+                            size_t workspace_bytes, void* stream);
 
 /* ---- sparse attend ([UGS] step 5; [Stem] Implementação) ------------------------- */
 

@@ -56,7 +56,7 @@ def test_workspace_sizes():
     s = _shape()
     n = bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_MEAN)
     nkb = 8 * 2048
-    assert n >= nkb * 128 * (4 + 2 + 2)
+    assert n >= nkb * 128 * (4 + 2) + nkb * 4          # fp32 pooled keys, fp16 copy, block scales
     n2 = bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_MEAN_VNORM)
     assert n2 >= n + nkb * 4
     p = bb.SelectParams(64, 64, 2, 0.25, float("nan"))
@@ -164,6 +164,44 @@ def test_score_kinds_validation():
     assert L.bsa_score_ex(ctypes.byref(s), bb.BSA_SCORE_KMINMAX, None, 16, 16, None, 16, None, 256,
                           n_mean, None) == bb.BSA_ERR_INVALID_ARG
     assert b"workspace" in L.bsa_last_error()
+
+
+def test_score_select_workspace_and_validation():
+    """bsa_score_select: workspace = score + selection workspaces + the ranking kernel's row
+    ring (fused shapes) or a scores array (the others); argument errors before any launch."""
+    L = bb.lib()
+    s = _shape()                                       # bf16, d 128, tiles of 128: fused
+    p = bb.SelectParams(64, 64, 2, 0.25, float("nan"))
+    n_sc = bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_MEAN)
+    n_sel = bb.bsa_select_workspace_bytes(s, p)
+    n = bb.bsa_score_select_workspace_bytes(s, bb.BSA_SCORE_MEAN, p)
+    assert n >= n_sc + n_sel + 2 * 2 * 2048 * 4
+    assert n < n_sc + n_sel + 32 * 1024 * 2048 * 4     # no scores array
+    # K-min/K-max and fp32 inputs run unfused: the scores pass through the workspace
+    nb = bb.bsa_score_select_workspace_bytes(s, bb.BSA_SCORE_KMINMAX, p)
+    assert nb >= bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_KMINMAX) + n_sel + 32 * 1024 * 2048 * 4
+    f = bb.Shape(1, 2, 2, 1024, 64, 64, 64, bb.BSA_F32)
+    pf = bb.SelectParams(4, 4, 1, 0.25, float("nan"))
+    nf = bb.bsa_score_select_workspace_bytes(f, bb.BSA_SCORE_MEAN, pf)
+    assert nf >= bb.bsa_select_workspace_bytes(f, pf) + 2 * 16 * 16 * 4
+    assert bb.bsa_score_select_workspace_bytes(s, 9, p) == 0
+    assert bb.bsa_score_select_workspace_bytes(s, bb.BSA_SCORE_MEAN, bb.SelectParams(0, 0, 1, 0.25, 0.0)) == 0
+    big = 1 << 36
+
+    def call(kind=bb.BSA_SCORE_MEAN, sp=None, prm=p, q=256, k=256, v=None, kv=256, cnt=256, ws=256,
+             wsb=big):
+        return L.bsa_score_select(ctypes.byref(s), kind, sp, ctypes.byref(prm), q, k, v, None, kv, cnt,
+                                  None, None, None, None, None, ws, wsb, None)
+    assert call(kv=None) == bb.BSA_ERR_INVALID_ARG
+    assert call(cnt=None) == bb.BSA_ERR_INVALID_ARG
+    assert call(ws=None) == bb.BSA_ERR_INVALID_ARG
+    assert call(q=None) == bb.BSA_ERR_INVALID_ARG
+    assert call(ws=272) == bb.BSA_ERR_INVALID_ARG and b"256-byte" in L.bsa_last_error()
+    assert call(q=264) == bb.BSA_ERR_INVALID_ARG and b"16-byte" in L.bsa_last_error()
+    assert call(wsb=n - 1) == bb.BSA_ERR_INVALID_ARG and b"workspace" in L.bsa_last_error()
+    assert call(kind=bb.BSA_SCORE_MEAN_VNORM) == bb.BSA_ERR_INVALID_ARG      # needs v
+    assert call(kind=bb.BSA_SCORE_MEAN_VLOG, v=256) == bb.BSA_ERR_INVALID_ARG  # needs beta
+    assert call(prm=bb.SelectParams(8, 9, 1, 0.25, 0.0)) == bb.BSA_ERR_INVALID_ARG
 
 
 def test_decode_list_validation():

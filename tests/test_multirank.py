@@ -85,13 +85,20 @@ def test_path_rooflines_closed_forms():
     spec = S.WORKLOADS[B.WORKLOAD]
     assert (spec.tile_q, spec.block_k) == (128, 64)
     n_qt, heads = spec.N // 128, spec.B * spec.Hq
-    r = B.path_rooflines(spec, 2.0, 0.5, {"bf16_tflops_sustained": 1000.0, "hbm_gbs": 5000.0})
+    r = B.path_rooflines(spec, 2.0, {"score_ms": 3.0, "select_ms": 0.5},
+                         {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0})
     flop = 2 * spec.d * 128 * heads * n_qt * (n_qt + 1)
-    assert r["score"]["algorithmic_tflop"] == pytest.approx(flop / 1e12)
-    assert r["score"]["tflops"] == pytest.approx(flop / 2e-3 / 1e12)
-    assert r["score"]["frac_tensor_sustained"] == pytest.approx(flop / 2e-3 / 1e12 / 1000.0)
+    f = r["score_select"]
+    assert f["algorithmic_tflop"] == pytest.approx(flop / 1e12)
+    assert f["tflops"] == pytest.approx(flop / 2e-3 / 1e12)
+    assert f["frac_tensor_burst"] == pytest.approx(flop / 2e-3 / 1e12 / 1000.0)
     q_k = (heads + spec.B * spec.Hkv) * spec.N * spec.d * 2
-    assert r["score"]["bytes"] == q_k + heads * n_qt * (n_qt + 1) * 4
     W = min(spec.rho * spec.k_first, spec.N // 64)
-    assert r["select"]["bytes"] == heads * n_qt * (n_qt - 1) * 4 + heads * n_qt * W * 4
-    assert r["select"]["frac_hbm"] == pytest.approx(r["select"]["bytes"] / 0.5e-3 / 1e9 / 5000.0)
+    assert f["bytes"] == q_k + heads * n_qt * (W + 1) * 4            # kv_idx and kv_cnt written
+    assert f["frac_hbm"] == pytest.approx(f["bytes"] / 2e-3 / 1e9 / 5000.0)
+    u = r["unfused"]
+    assert u["score_tflops"] == pytest.approx(flop / 3e-3 / 1e12)
+    assert u["score_GBps"] == pytest.approx((q_k + heads * n_qt * (n_qt + 1) * 4) / 3e-3 / 1e9)
+    sel = heads * n_qt * (n_qt - 1) * 4 + heads * n_qt * W * 4
+    assert u["select_GBps"] == pytest.approx(sel / 0.5e-3 / 1e9)
+    assert u["select_frac_hbm"] == pytest.approx(sel / 0.5e-3 / 1e9 / 5000.0)
