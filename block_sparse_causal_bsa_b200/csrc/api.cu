@@ -231,7 +231,7 @@ bsa_status run_gate_finalize(const bsa_shape& s, const bsa_select_params& p, int
 struct ScoreSelectWs {
   ScoreWs sc;
   SelectWs sel;
-  float* ring;       // fused: [kScoreRankRingCtas][2][heads per unit][n_kb]
+  float* ring;       // fused: [kScoreRankRingCtas][kScoreRankRing][heads per unit][n_kb]
   float* scores;     // unfused: [B,Hq,n_qt,n_kb]
   size_t bytes;
 };
@@ -248,9 +248,10 @@ ScoreSelectWs score_select_ws(const bsa_shape& s, bsa_score_kind kind, int W, vo
   w.sel = select_ws(s, W, p ? p + off : nullptr);
   off += w.sel.bytes;
   const size_t n_kb = (size_t)(s.N / s.block_k);
-  if (fused_kind(kind) && bsa::score_rank_supported(s)) {
+  if (fused_kind(kind) && bsa::score_rank_fusable(s)) {
     w.ring = (float*)(p + off);
-    off += align256((size_t)bsa::kScoreRankRingCtas * 2 * bsa::score_rank_heads_per_unit(s) * n_kb * 4);
+    off += align256((size_t)bsa::kScoreRankRingCtas * bsa::kScoreRankRing *
+                    bsa::score_rank_heads_per_unit(s) * n_kb * 4);
   } else {
     w.scores = (float*)(p + off);
     off += align256((size_t)s.B * s.Hq * (s.N / s.tile_q) * n_kb * 4);

@@ -40,10 +40,13 @@ cudaError_t launch_score_tc_bounds(const bsa_shape& s, const void* q, const uint
 // optionally fused with the ranking of the selection. kbar16/kinv from launch_pool.
 // ranked == null: scores only (scores required). ranked != null: also the top-M lists
 // [B*Hq*n_qt][W] and sigma; scores may then be null, and the rows go through
-// ring [ring_ctas][2][heads per unit][n_kb] instead (the grid is capped at ring_ctas).
+// ring [ring_ctas][kScoreRankRing][heads per unit][n_kb] instead (the grid is capped at
+// ring_ctas).
 bool score_rank_supported(const bsa_shape& s);
+bool score_rank_fusable(const bsa_shape& s);          // the ranking too
 int score_rank_heads_per_unit(const bsa_shape& s);
 constexpr int kScoreRankRingCtas = 256;
+constexpr int kScoreRankRing = 8;
 cudaError_t launch_score_rank(const bsa_shape& s, const bsa_select_params* p, const void* q,
                               const uint16_t* kbar16, const float* kinv, const float* wnorm, int wmode,
                               float* scores, float* ring, int ring_ctas, int32_t* ranked, float* sigma,

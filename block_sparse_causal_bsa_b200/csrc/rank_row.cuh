@@ -457,4 +457,5 @@ __device__ float rank_row(const float* s, int n, const TileSlots& sl, float xmin
   return sg;
 }
 
+
 }  // namespace bsa

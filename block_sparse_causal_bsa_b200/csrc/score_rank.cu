@@ -28,9 +28,11 @@
 //                   of its unit; per chunk, the row max from TMEM, the exact rescale,
 //                   the value term, and the row written to the scores array or to an
 //                   L2-resident ring; per unit, the row's min / max / finiteness.
-//   6.. (RANK)      one rank warp per head: ranks the finished row (rank_row) while
-//                   the tensor cores score the next unit, writes the top-M list with
-//                   the top-m flag and sigma.
+//   6-10 (RANK)     five rank warps: each ranks whole rows (rank_row), rows taken in
+//                   unit order round-robin, reading the row from L2 in every pass, while
+//                   the tensor cores score later units; writes the top-M list with the
+//                   top-m flag and sigma. The rows of up to 8 units wait in the ring, so
+//                   the epilogue runs ahead of the ranking.
 // Every wait is bounded (tc::mbar_wait); a timeout raises BSA_DEV_TIMEOUT and the CTA
 // unwinds, waits for its own copies and MMAs, and frees its TMEM.
 // Shapes: bf16 inputs, d = 128, query tile 128, key block 64 or 128.
@@ -52,9 +54,12 @@ constexpr int kEpiWarps = 4;
 constexpr uint32_t kHalfTile = 16384;         // 128 rows x 128 bytes: one 64-column half
 constexpr uint32_t kChunk = 2 * kHalfTile;    // one pooled-key chunk (128 blocks x 128 dims, fp16)
 
+constexpr int kRankWarpsF = 5;                // rank warps of the fused kernel
+constexpr int kRing = kScoreRankRing;         // units whose rows the L2 ring holds
+
 template <int HP, bool RANK>
 struct SRLayout {
-  static constexpr int rank_warps = RANK ? HP : 0;
+  static constexpr int rank_warps = RANK ? kRankWarpsF : 0;
   static constexpr int threads = (2 + kEpiWarps + rank_warps) * 32;
   static constexpr uint32_t qhalf = HP * kHalfTile;     // one d-half of all HP heads' tiles
   static constexpr uint32_t qbuf = 2 * qhalf;           // one Q buffer
@@ -76,13 +81,13 @@ struct __align__(8) SRCtrl {
   uint64_t q_full[2], qc_full[2], q_empty[2];
   uint64_t kb_full[2], kb_empty[2];
   uint64_t d_full[2], d_free[2];
-  uint64_t row_full[2], row_free[2];
+  uint64_t row_full[kRing], row_free[kRing];
   uint64_t qmax_bar;
   uint64_t done;
   uint32_t tmem;
   int abort_flag;
   uint32_t qmax_part[2][HP][kEpiWarps];   // by phase parity of qmax_bar, head, epilogue warp
-  RowStat stat[2][HP][kEpiWarps]; // per row slot, head, epilogue warp
+  RowStat stat[kRing][HP][kEpiWarps];     // per ring slot, head, epilogue warp
 };
 
 __device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
@@ -105,7 +110,7 @@ struct SRArgs {
   const float* wnorm;     // value term per block, or null
   int wmode;              // 0 none, 1 times w, 2 plus w
   float* scores;          // [B,Hq,n_qt,n_kb] or null (ranking only)
-  float* ring;            // [grid][2][HP][n_kb] when scores is null
+  float* ring;            // [grid][kRing][HP][n_kb] when scores is null
   int32_t* ranked;        // [B*Hq*n_qt][W] top-M lists (ranking)
   float* sigma;           // [B*Hq*n_qt]
   int W;
@@ -149,6 +154,8 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
       tc::mbar_init(&c.kb_empty[i], 1);
       tc::mbar_init(&c.d_full[i], 1);
       tc::mbar_init(&c.d_free[i], kEpiWarps);
+    }
+    for (int i = 0; i < kRing; ++i) {
       tc::mbar_init(&c.row_full[i], kEpiWarps);
       tc::mbar_init(&c.row_free[i], HP);
     }
@@ -322,7 +329,7 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
     bool ok = (int)blockIdx.x >= a.units || convert(0);
     int gc = 0;
     for (int li = 0, u = blockIdx.x; ok && u < a.units; ++li, u += stride) {
-      const int slot = li & 1, qb = li & 1;
+      const int slot = li % kRing, qb = li & 1;
       int t, bg, pr;
       unit_coords(u, npair, BG, a.n_qt, t, bg, pr);
       const int b = bg / a.Hkv, g = bg % a.Hkv;
@@ -332,8 +339,8 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
       const int nc = (J + 1 + CB - 1) / CB;
       const bool next = u + stride < a.units;
       const int conv_at = nc - 1 < 3 ? nc - 1 : 3;    // chunk before which the next Q is converted
-      if (RANK && li >= 2 &&
-          !warp_all(tc::mbar_wait(&c.row_free[slot], ((li >> 1) - 1) & 1, abort_flag, dev_status))) {
+      if (RANK && li >= kRing &&
+          !warp_all(tc::mbar_wait(&c.row_free[slot], (li / kRing - 1) & 1, abort_flag, dev_status))) {
         ok = false;
         break;
       }
@@ -341,7 +348,7 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
 #pragma unroll
       for (int hp = 0; hp < HP; ++hp)
         rows[hp] = a.scores ? a.scores + (((size_t)b * a.Hq + h0 + hp) * a.n_qt + t) * a.n_kb
-                            : a.ring + (((size_t)blockIdx.x * 2 + slot) * HP + hp) * a.n_kb;
+                            : a.ring + (((size_t)blockIdx.x * kRing + slot) * HP + hp) * a.n_kb;
       float mn[HP], mxv[HP];
       bool bad[HP];
 #pragma unroll
@@ -361,13 +368,30 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
         tc::tc_fence_after();
 #pragma unroll
         for (int hp = 0; hp < HP; ++hp) {
-          float m = -INFINITY;
+          float m;
+          if constexpr (RANK) {
+            // 32 columns per load: the rank warps leave 168 registers per thread
+            m = -INFINITY;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t v[32];
-            tc::tmem_ld32(tl + db * L::dcols + hp * TQ + cc * 32, v);
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t v[32];
+              tc::tmem_ld32(tl + db * L::dcols + hp * TQ + cc * 32, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) m = fmaxf(m, __uint_as_float(v[i]));
+              for (int i = 0; i < 32; ++i) m = fmaxf(m, __uint_as_float(v[i]));
+            }
+          } else {
+            float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              uint32_t v[64];
+              tc::tmem_ld64(tl + db * L::dcols + hp * TQ + cc * 64, v);
+#pragma unroll
+              for (int i = 0; i < 64; i += 2) {
+                m0 = fmaxf(m0, __uint_as_float(v[i]));
+                m1 = fmaxf(m1, __uint_as_float(v[i + 1]));
+              }
+            }
+            m = fmaxf(m0, m1);
           }
           float val = (m * qi[hp]) * kv;             // exact: powers of two
           if (a.wmode == 1) val = val * wv;
@@ -403,34 +427,39 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
       }
     }
   } else if (RANK && warp >= 2 + kEpiWarps) {
-    // ---------------- rank warps: one per head of the unit ----------------
-    const int hp = warp - (2 + kEpiWarps);
-    uint32_t* slice = reinterpret_cast<uint32_t*>(sm + L::smem_rank) + (size_t)hp * kRankSliceWords;
-    for (int li = 0, u = blockIdx.x; u < a.units; ++li, u += stride) {
-      const int slot = li & 1;
-      if (!warp_all(tc::mbar_wait(&c.row_full[slot], (li >> 1) & 1, abort_flag, dev_status))) break;
+    // ---------------- rank warps ----------------
+    // Rows are numbered in unit order (row li*HP + hp); rank warp w takes the rows congruent
+    // to w modulo kRankWarpsF, so several rows are ranked at once while the tensor cores
+    // score later units. A warp reads its row from L2 (the ring, or the scores array) in
+    // every ranking pass; the ring slot is freed when the unit's HP rows are ranked.
+    const int rw = warp - (2 + kEpiWarps);
+    uint32_t* slice = reinterpret_cast<uint32_t*>(sm + L::smem_rank) + (size_t)rw * kRankSliceWords;
+    const int li_end = ((int)a.units - (int)blockIdx.x + stride - 1) / stride;   // units of this CTA
+    for (int gr = rw; gr < li_end * HP; gr += kRankWarpsF) {
+      const int li = gr / HP, hp = gr % HP;
+      const int slot = li % kRing;
+      if (!warp_all(tc::mbar_wait(&c.row_full[slot], (li / kRing) & 1, abort_flag, dev_status))) break;
+      const int u = blockIdx.x + li * stride;
       int t, bg, pr;
       unit_coords(u, npair, BG, a.n_qt, t, bg, pr);
       const int b = bg / a.Hkv, g = bg % a.Hkv;
-      const int h = g * G + pr * HP + hp;
-      const size_t row = ((size_t)b * a.Hq + h) * a.n_qt + t;
+      const size_t row = ((size_t)b * a.Hq + g * G + pr * HP + hp) * a.n_qt + t;
       const TileSlots sl = tile_slots(t, a.n_qt, TQ, a.block_k, a.k_first, a.k_last, a.rho);
       const int n = sl.f_lo;
-      float sg = 1.0f;
-      bool bad = false;
-      if (n > 0) {
-        float xmin = c.stat[slot][hp][0].mn, xmax = c.stat[slot][hp][0].mx;
-        int anybad = c.stat[slot][hp][0].bad;
+      float xmin = c.stat[slot][hp][0].mn, xmax = c.stat[slot][hp][0].mx;
+      int anybad = c.stat[slot][hp][0].bad;
 #pragma unroll
-        for (int w = 1; w < kEpiWarps; ++w) {
-          xmin = fminf(xmin, c.stat[slot][hp][w].mn);
-          xmax = fmaxf(xmax, c.stat[slot][hp][w].mx);
-          anybad |= c.stat[slot][hp][w].bad;
-        }
-        bad = anybad != 0;
-        const float* s = a.scores ? a.scores + row * a.n_kb
-                                  : a.ring + (((size_t)blockIdx.x * 2 + slot) * HP + hp) * a.n_kb;
-        sg = rank_row<false>(s, n, sl, xmin, xmax, bad, slice, a.ranked + row * a.W, lane);
+      for (int w = 1; w < kEpiWarps; ++w) {
+        xmin = fminf(xmin, c.stat[slot][hp][w].mn);
+        xmax = fmaxf(xmax, c.stat[slot][hp][w].mx);
+        anybad |= c.stat[slot][hp][w].bad;
+      }
+      const bool bad = n > 0 && anybad != 0;
+      float sg = 1.0f;
+      if (n > 0) {
+        const float* src = a.scores ? a.scores + row * a.n_kb
+                                    : a.ring + (((size_t)blockIdx.x * kRing + slot) * HP + hp) * a.n_kb;
+        sg = rank_row<false>(src, n, sl, xmin, xmax, bad, slice, a.ranked + row * a.W, lane);
       }
       if (lane == 0) {
         if (bad) {
@@ -470,6 +499,8 @@ bool score_rank_supported(const bsa_shape& s) {
          (long long)s.B * s.Hq * s.N < (1ll << 31) &&
          (long long)s.B * s.Hkv * (s.N / s.block_k) < (1ll << 31);
 }
+
+bool score_rank_fusable(const bsa_shape& s) { return score_rank_supported(s); }
 
 int score_rank_heads_per_unit(const bsa_shape& s) { return ((s.Hq / s.Hkv) % 2 == 0) ? 2 : 1; }
 

@@ -80,6 +80,13 @@ def test_fused_key_blocks_of_128():
     _case(spec, 2103)
 
 
+def test_fused_rows_not_16_byte_aligned():
+    # n_kb = 74: score rows start on 8-byte boundaries, so the rank warps copy them one
+    # element at a time
+    spec = S.WORKLOADS["gated_prefill_128k"].scaled(N=128 * 37, Hq=8, Hkv=2, k_first=12, k_last=12)
+    _case(spec, 2108)
+
+
 @pytest.mark.parametrize("kind,beta", [("vnorm", 0.0), ("vlog", 0.5)])
 def test_fused_output_aware_with_budget_decay(kind, beta):
     spec = S.WORKLOADS["tpd_oam_prefill_64k"].scaled(N=8192, Hq=8, Hkv=2, B=2, k_first=32, k_last=8)
