@@ -15,49 +15,29 @@
 // must order them. Nothing in it has to start at zero (the selection kernels
 // write every scratch entry they later read), and it keeps whatever the last
 // call left there.
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 
 namespace {
 
 constexpr size_t kSelectScratchBytes = size_t(32) << 20;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_select_scratch[kSelectScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_select_scratch on the current device. In host code the
-// name g_select_scratch is only a host-side stand-in for the symbol, never a
-// device address, so the address is looked up once per device (with that
-// device current) and cached.
+// Device address of g_select_scratch in the current device's current context. In host
+// code the name g_select_scratch is only a host-side stand-in for the symbol, never a
+// device address, so the address is looked up with the device current. It is looked up
+// on every call (a host-side table lookup once the module is loaded): an address cached
+// across calls could go stale after cudaDeviceReset, or belong to another context made
+// current on the same device.
 bsa_status scratch_for_current_device(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) {
-    bsa::set_last_error("bsa_select_noalloc: cudaGetDevice failed: %s", cudaGetErrorString(e));
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_select_scratch);
+  if (e != cudaSuccess || !p) {
+    bsa::set_last_error("bsa_select_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
     return BSA_ERR_CUDA;
   }
-  if (dev < 0 || dev >= kMaxDevices) {
-    bsa::set_last_error("bsa_select_noalloc: device %d beyond the %d devices tracked", dev,
-                        kMaxDevices);
-    return BSA_ERR_UNSUPPORTED;
-  }
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_select_scratch);
-    if (e != cudaSuccess || !p) {
-      bsa::set_last_error("bsa_select_noalloc: cudaGetSymbolAddress failed: %s",
-                          cudaGetErrorString(e));
-      return BSA_ERR_CUDA;
-    }
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return BSA_OK;
 }
 

@@ -321,8 +321,9 @@ bsa_status bsa_decode_list(const bsa_decode_shape* shape, const bsa_decode_param
  * every GPU loading libbsa.so keeps until the process exits.
  *   - Shapes whose bsa_select_workspace_bytes() exceed that size are rejected with
  *     BSA_ERR_UNSUPPORTED (bsa_last_error() says why); nothing is launched.
- *   - The first call on a device looks up the array's device address (with that
- *     device current) and caches it; make that first call before any stream capture.
+ *   - Every call looks up the array's device address in the current device's
+ *     current context. The first call on a device also loads the library's device
+ *     code there; make that first call before any stream capture.
  *   - All calls share the one array. Calls that overlap on the GPU (other streams,
  *     other host threads on the same device) race on it: the caller must order them.
  *     The array keeps the last call's contents; no entry has to start at zero. */

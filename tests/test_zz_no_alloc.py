@@ -87,6 +87,51 @@ def test_noalloc_matches_workspace_path_twice():
     assert not torch.equal(first["kv_cnt"], second["kv_cnt"])
 
 
+def test_noalloc_without_optional_outputs():
+    """sigma, sigma_bar and trigger NULL: the call then keeps them in the static scratch's
+    own regions, and kv_idx, kv_cnt and theta must still match bsa_select bit for bit."""
+    shape, params, scores = _case(3003, 10)
+    L = bb.lib()
+    W = bb.bsa_kv_idx_width(shape, params)
+    B, Hq, n_qt, _ = scores.shape
+    ref = _outputs(B, Hq, n_qt, W)
+    got = _outputs(B, Hq, n_qt, W)
+    nb = bb.bsa_select_workspace_bytes(shape, params)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    for _ in range(2):                               # twice: the second call finds stale scratch
+        st = L.bsa_select(ctypes.byref(shape), ctypes.byref(params), scores.data_ptr(),
+                          ref["kv_idx"].data_ptr(), ref["kv_cnt"].data_ptr(), None, None, None,
+                          ref["theta"].data_ptr(), ref["dev_status"].data_ptr(), ws.data_ptr(), nb,
+                          stream)
+        assert st == bb.BSA_OK, L.bsa_last_error()
+        st = L.bsa_select_noalloc(ctypes.byref(shape), ctypes.byref(params), scores.data_ptr(),
+                                  got["kv_idx"].data_ptr(), got["kv_cnt"].data_ptr(), None, None, None,
+                                  got["theta"].data_ptr(), got["dev_status"].data_ptr(), stream)
+        assert st == bb.BSA_OK, L.bsa_last_error()
+        torch.cuda.synchronize()
+        for key in ("kv_idx", "kv_cnt", "dev_status"):
+            assert torch.equal(ref[key], got[key]), key
+        assert torch.equal(ref["theta"].view(torch.int32), got["theta"].view(torch.int32))
+    assert int(got["dev_status"].item()) == 0
+
+
+def test_noalloc_shape_just_under_the_limit():
+    """A layer whose selection workspace fills 99 % of the static scratch (63 query heads
+    at 128k, W = 128): the call accepts it and matches bsa_select. Scores are random
+    (the selection reads any finite scores)."""
+    L = bb.lib()
+    limit = L.bsa_select_noalloc_max_bytes()
+    shape = bb.Shape(1, 63, 7, 131072, 128, 64, 128, bb.BSA_BF16)
+    params = bb.SelectParams(64, 64, 2, 0.25, float("nan"))
+    need = bb.bsa_select_workspace_bytes(shape, params)
+    assert 0.98 * limit < need <= limit
+    g = torch.Generator(device="cuda").manual_seed(3004)
+    scores = torch.randn(1, 63, 1024, 2048, device="cuda", generator=g)
+    _run_both(shape, params, scores)
+    del scores
+
+
 def test_noalloc_rejects_oversized_shapes():
     L = bb.lib()
     limit = L.bsa_select_noalloc_max_bytes()
