@@ -240,6 +240,105 @@ def cpu_baseline(spec, seed, target_s=15.0):
                       f"{dt:.1f} s, selected-block flops / time"}
 
 
+def _causal_score_flops(spec):
+    """Algorithmic block-score flops of a whole layer: 2 * d * tile_q per (b, h, tile, causal block)."""
+    n_qt = spec.N // spec.tile_q
+    causal = sum(((t + 1) * spec.tile_q - 1) // spec.block_k + 1 for t in range(n_qt))
+    return 2.0 * spec.d * spec.tile_q * causal * spec.B * spec.Hq
+
+
+def cpu_config_baselines(n_rows_c4=192, n_groups_c5=6):
+    """The oracle timed per workload on the host cores, in the unit of the matching GPU
+    figure (bounded samples where a whole layer would take minutes). Input generation is
+    outside the timed region. Returns {workload: entry}."""
+    from block_sparse_causal_bsa_b200 import synthetic as S
+    from oracle import bsa_oracle as O
+    cores, host = _blas_threads(), os.cpu_count()
+    out = {}
+
+    def entry(value, unit, dt, sample):
+        return {"value": value, "unit": unit, "cores": cores, "host_cpus": host, "kind": "oracle",
+                "seconds": dt, "sample": sample}
+
+    # tiny fp32: the whole path (scores, selection, attend)
+    spec = S.WORKLOADS["tiny_fp32_1k"]
+    q, k, v = S.prefill_inputs(spec, 1001)
+    t0 = time.perf_counter()
+    sc = O.block_scores(q, k, spec.tile_q, spec.block_k)
+    sel = O.select(sc, spec.tile_q, spec.block_k, spec.k_first, spec.k_last, spec.rho, spec.gate_quantile)
+    O.attend(q, k, v, sel["kv_idx"], spec.tile_q, spec.block_k, 1.0 / math.sqrt(spec.d))
+    dt = time.perf_counter() - t0
+    fl = 4.0 * spec.tile_q * spec.block_k * spec.d * float(sel["kv_cnt"].sum())
+    out[spec.name] = entry(fl / dt / 1e12, "TFLOP/s", dt, "the whole problem: scores, selection and "
+                           "attend of every tile; selected-block flops / time")
+    # 32k vertical-slash workload: scores and selection of the whole layer
+    spec = S.WORKLOADS["prefill_32k_vs"]
+    q, k, _ = S.prefill_inputs(spec, 1002)
+    t0 = time.perf_counter()
+    sc = O.block_scores(q, k, spec.tile_q, spec.block_k)
+    O.select(sc, spec.tile_q, spec.block_k, spec.k_first, spec.k_last, spec.rho, spec.gate_quantile)
+    dt = time.perf_counter() - t0
+    out[spec.name] = entry(_causal_score_flops(spec) / dt / 1e12, "TFLOP/s", dt,
+                           "scores and selection of the whole layer; algorithmic score flops / time")
+    del q, k, sc
+    # 64k position-decay budget, output-aware score: a seeded sample of (b, h, tile) rows
+    spec = S.WORKLOADS["tpd_oam_prefill_64k"]
+    rng = np.random.default_rng(11)
+    G = spec.Hq // spec.Hkv
+    rows = [(int(rng.integers(spec.B)), int(rng.integers(spec.Hq)), int(rng.integers(spec.n_qt)))
+            for _ in range(n_rows_c4)]
+    data = {}
+    for b, h, _ in rows:
+        for name, hh in (("q", h), ("k", h // G), ("v", h // G)):
+            if (name, b, hh) not in data:
+                data[name, b, hh] = S.prefill_head(spec, 1004, name, b, hh)
+    t0 = time.perf_counter()
+    pooled = {}
+    fl = 0.0
+    sig = []
+    for b, h, t in rows:
+        g = h // G
+        if (b, g) not in pooled:
+            pooled[b, g] = (O.pool_keys(data["k", b, g], spec.block_k),
+                            O.value_block_norm(data["v", b, g], spec.block_k))
+        kbar, w = pooled[b, g]
+        f_lo, J = O.tile_blocks(t, spec.tile_q, spec.block_k)
+        row = O.score_tile(data["q", b, h][t * spec.tile_q:(t + 1) * spec.tile_q], kbar, J, w)
+        nF, nc, m, M = O.tile_slots(t, spec.n_qt, spec.tile_q, spec.block_k, spec.k_first, spec.k_last,
+                                    spec.rho)
+        order = O.rank_candidates(row, nc)
+        if nc > m >= 1:
+            sig.append(O.cut_margin(row, order, m))
+        fl += 2.0 * spec.d * spec.tile_q * (J + 1)
+    dt = time.perf_counter() - t0
+    out[spec.name] = entry(fl / dt / 1e12, "TFLOP/s", dt,
+                           f"{n_rows_c4} random (b,h,t) rows: pooling of their KV heads (keys and "
+                           "value norms), output-aware scores, ranking and sigma; score flops / time")
+    del data, pooled
+    # decode with run-time termination: a sample of (batch, KV head) groups
+    dspec = S.DECODE_WORKLOADS["decode_art_64k"]
+    G = dspec.Hq // dspec.Hkv
+    dims = S.default_probe_dims(32)
+    groups = [(int(b), int(g)) for b, g in zip(rng.integers(dspec.B, size=n_groups_c5),
+                                               rng.integers(dspec.Hkv, size=n_groups_c5))]
+    ins = {(b, g): (np.stack([S.decode_head(dspec, 2005, "q", b, g * G + i) for i in range(G)]),
+                    S.decode_head(dspec, 2005, "k", b, g), S.decode_head(dspec, 2005, "v", b, g))
+           for b, g in groups}
+    t0 = time.perf_counter()
+    used = 0
+    for b, g in groups:
+        qg, kc, vc = ins[b, g]
+        _, u, _ = O.decode_group(qg, kc, vc, dspec.block_kv, 1.0 / math.sqrt(dspec.d), dspec.tau,
+                                 dspec.phi, dspec.patience, dims)
+        used += u
+    dt = time.perf_counter() - t0
+    byts = used * dspec.block_kv * dspec.d * 2 * 2
+    out[dspec.name] = entry(byts / dt / 1e9, "GB/s", dt,
+                            f"{n_groups_c5} random (batch, KV head) groups with termination on; KV bytes "
+                            "of the blocks used / time (the oracle forms every block's partial output)")
+    return out
+
+
 # ---------------------------------------------------------------------------
 # GPU arm
 
@@ -295,6 +394,10 @@ def main_gpu(args):
     cfg = bb.SelectConfig(spec.k_first, spec.k_last, spec.rho, spec.gate_quantile)
     prm = cfg.c()
     W = bb.bsa_kv_idx_width(shape, prm)
+    paths = {"score_select": bb.bsa_score_path(shape, bb.BSA_SCORE_MEAN),
+             "attend": bb.bsa_attend_path(shape, W)}
+    if any(v != bb.BSA_PATH_TENSOR_CORES for v in paths.values()):
+        raise RuntimeError(f"the benchmark shape would leave the tensor cores: {paths}")
     B, Hq, N, d = q.shape
     n_qt, n_kb = N // spec.tile_q, N // spec.block_k
     scores = torch.empty(B, Hq, n_qt, n_kb, dtype=torch.float32, device=dev)
@@ -314,6 +417,23 @@ def main_gpu(args):
     ws_f = torch.empty(ws_f_n, dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     scale = 1.0 / math.sqrt(d)
+
+    def time_call(fn, reps=5, status=None):
+        """Mean device time (ms) of fn over reps calls, L2 flushed before each."""
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            fn()
+            b_.record(stream)
+            ts.append((a_, b_))
+        torch.cuda.synchronize()
+        if status is not None and int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item())}")
+        return statistics.mean(a_.elapsed_time(b_) for a_, b_ in ts)
 
     def step(q_, k_, v_, out_, ev=None):
         # scores and selection in one call (the ranking runs inside the score kernel; the
@@ -519,7 +639,58 @@ def main_gpu(args):
               "ms": vs_ms, "visited_block_pairs": visited,
               "visited_fraction_of_causal": visited / (vspec.B * vspec.Hq * sum(2 * t + 2 for t in range(vspec.N // 128))),
               "executed_tflops": vs_flops / (vs_ms * 1e-3) / 1e12}
-    del vq, vk, vv, vws, vout
+    # the same workload's scores and selection (one fused call, scores not written out)
+    vcfg = bb.SelectConfig(vspec.k_first, vspec.k_last, vspec.rho, vspec.gate_quantile)
+    vsel = {}
+
+    def run_vsel():
+        vsel["r"] = bb.score_select(vq, vk, None, block_k=vspec.block_k, tile_q=vspec.tile_q, cfg=vcfg,
+                                    want_scores=False)
+    ms_c2 = time_call(run_vsel)
+    if int(vsel["r"]["dev_status"].item()) != 0:
+        raise RuntimeError("32k score/select: device status")
+    gpu_configs = {vspec.name: {"value": _causal_score_flops(vspec) / (ms_c2 * 1e-3) / 1e12,
+                                "unit": "TFLOP/s", "ms": ms_c2,
+                                "scope": "scores and selection of the whole layer (bsa_score_select); "
+                                         "algorithmic score flops / time"}}
+    del vq, vk, vv, vws, vout, vsel
+
+    # the tiny fp32 workload: the whole path (fp32 CUDA-core kernels)
+    tspec = S.WORKLOADS["tiny_fp32_1k"]
+    tq, tk, tv = (torch.from_numpy(x).to(dev) for x in S.prefill_inputs(tspec, 1001))
+    tcfg = bb.SelectConfig(tspec.k_first, tspec.k_last, tspec.rho, tspec.gate_quantile)
+    tres = {}
+
+    def run_tiny():
+        tres["r"] = bb.prefill(tq, tk, tv, block_k=tspec.block_k, tile_q=tspec.tile_q, cfg=tcfg)
+    ms_c1 = time_call(run_tiny)
+    t_out, t_sel, t_st = tres["r"]
+    if int(t_st.item()) != 0 or int(t_sel["dev_status"].item()) != 0:
+        raise RuntimeError("tiny fp32 prefill: device status")
+    gpu_configs[tspec.name] = {"value": 4.0 * tspec.tile_q * tspec.block_k * tspec.d * float(t_sel["kv_cnt"].sum())
+                               / (ms_c1 * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms_c1,
+                               "scope": "the whole path (scores and selection, attend); selected-block "
+                                        "flops / time"}
+    del tq, tk, tv, tres, t_out, t_sel
+
+    # the 64k position-decay, output-aware workload: scores and selection (fused call)
+    cspec = S.WORKLOADS["tpd_oam_prefill_64k"]
+    cq, ck, cv = (_bf16(torch, x, dev) for x in _gen_prefill(cspec, 1004 + 1000 * rank))
+    ccfg = bb.SelectConfig(cspec.k_first, cspec.k_last, cspec.rho, cspec.gate_quantile)
+    cres = {}
+
+    def run_c4():
+        cres["r"] = bb.score_select(cq, ck, cv, block_k=cspec.block_k, tile_q=cspec.tile_q, cfg=ccfg,
+                                    kind="vnorm", want_scores=False)
+    ms_c4 = time_call(run_c4)
+    if int(cres["r"]["dev_status"].item()) != 0:
+        raise RuntimeError("64k score/select: device status")
+    gpu_configs[cspec.name] = {"value": _causal_score_flops(cspec) / (ms_c4 * 1e-3) / 1e12,
+                               "unit": "TFLOP/s", "ms": ms_c4,
+                               "scope": "scores (times the value-block norms) and selection with the "
+                                        "position-decay budget (bsa_score_select); algorithmic score "
+                                        "flops / time"}
+    del cq, ck, cv, cres
 
     # decode with run-time termination (timed on its own)
     dspec = S.DECODE_WORKLOADS[DECODE_WORKLOAD]
@@ -527,6 +698,9 @@ def main_gpu(args):
     dq, dk, dv = _bf16(torch, dq, dev), _bf16(torch, dk, dev), _bf16(torch, dv, dev)
     dims = S.default_probe_dims(32)
     dshape = bb.DecodeShape(dspec.B, dspec.Hq, dspec.Hkv, dspec.L, dspec.d, dspec.block_kv, bb.BSA_BF16)
+    paths["decode"] = bb.bsa_decode_path(dshape)
+    if paths["decode"] != bb.BSA_PATH_TENSOR_CORES:
+        raise RuntimeError("the decode workload would leave the tensor cores")
     cdims = (ctypes.c_int * len(dims))(*[int(x) for x in dims])
     dout = torch.empty_like(dq)
     used = torch.empty(dspec.B, dspec.Hkv, dtype=torch.int32, device=dev)
@@ -645,8 +819,20 @@ def main_gpu(args):
             "clocks": clocks,
             "decode": dec,
         }
+        gpu_configs[DECODE_WORKLOAD] = {"value": dec["terminated"]["GBps"], "unit": "GB/s",
+                                        "ms": dec["terminated"]["ms"],
+                                        "scope": "decode with termination on; KV bytes of the blocks "
+                                                 "used / time"}
+        gpu_configs[WORKLOAD] = {"value": res["value"], "unit": "TFLOP/s", "ms": step_ms,
+                                 "scope": "the headline step"}
+        res["kernel_paths"] = {k_: ("tensor cores" if v_ == bb.BSA_PATH_TENSOR_CORES else "CUDA cores")
+                               for k_, v_ in paths.items()}
+        res["configs"] = {name: {"gpu": g} for name, g in gpu_configs.items()}
         if world == 1 and not args.no_cpu:
             res["cpu_baseline"] = cpu_baseline(spec, seed)
+            res["configs"][WORKLOAD]["cpu_baseline"] = res["cpu_baseline"]
+            for name, e in cpu_config_baselines().items():
+                res["configs"][name]["cpu_baseline"] = e
         print(json.dumps(res), flush=True)
     if world > 1:
         dist.barrier()

@@ -26,6 +26,7 @@ BSA_OK, BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA = 0, 1, 2, 3
 BSA_DEV_OK, BSA_DEV_BAD_INDEX, BSA_DEV_TIMEOUT, BSA_DEV_BAD_SCORE = 0, 1, 2, 4
 BSA_BF16, BSA_F32 = 0, 1
 BSA_SCORE_MEAN, BSA_SCORE_MEAN_VNORM, BSA_SCORE_MEAN_VLOG, BSA_SCORE_KMINMAX = 0, 1, 2, 3
+BSA_PATH_CUDA_CORES, BSA_PATH_TENSOR_CORES = 0, 1
 SCORE_KINDS = {"mean": BSA_SCORE_MEAN, "vnorm": BSA_SCORE_MEAN_VNORM, "vlog": BSA_SCORE_MEAN_VLOG,
                "kminmax": BSA_SCORE_KMINMAX}
 
@@ -34,7 +35,7 @@ EXPORTS = ("bsa_score_workspace_bytes", "bsa_score", "bsa_kv_idx_width",
            "bsa_status_string", "bsa_last_error", "bsa_select_noalloc_max_bytes",
            "bsa_select_noalloc", "bsa_selftest_wait", "bsa_decode_list", "bsa_score_ex",
            "bsa_attend_vs_workspace_bytes", "bsa_attend_vs", "bsa_score_select_workspace_bytes",
-           "bsa_score_select")
+           "bsa_score_select", "bsa_score_path", "bsa_attend_path", "bsa_decode_path")
 
 
 class BsaError(RuntimeError):
@@ -120,6 +121,12 @@ def lib() -> ctypes.CDLL:
         L.bsa_attend_vs.restype = ctypes.c_int
         L.bsa_selftest_wait.argtypes = [ctypes.c_int, i32p, i32p, vp]
         L.bsa_selftest_wait.restype = ctypes.c_int
+        L.bsa_score_path.argtypes = [sp, ctypes.c_int]
+        L.bsa_score_path.restype = ctypes.c_int
+        L.bsa_attend_path.argtypes = [sp, ctypes.c_int]
+        L.bsa_attend_path.restype = ctypes.c_int
+        L.bsa_decode_path.argtypes = [dsp]
+        L.bsa_decode_path.restype = ctypes.c_int
         L.bsa_status_string.argtypes = [ctypes.c_int]
         L.bsa_status_string.restype = ctypes.c_char_p
         L.bsa_last_error.argtypes = []
@@ -230,6 +237,18 @@ def bsa_select_noalloc(shape, params, scores, kv_idx, kv_cnt, sigma, sigma_bar, 
                                     _ptr(kv_idx), _ptr(kv_cnt), _ptr(sigma), _ptr(sigma_bar),
                                     _ptr(trigger), _ptr(theta), _ptr(dev_status),
                                     _stream(stream)))
+
+
+def bsa_score_path(shape: Shape, kind: int) -> int:
+    return lib().bsa_score_path(ctypes.byref(shape), kind)
+
+
+def bsa_attend_path(shape: Shape, W: int) -> int:
+    return lib().bsa_attend_path(ctypes.byref(shape), int(W))
+
+
+def bsa_decode_path(shape: DecodeShape) -> int:
+    return lib().bsa_decode_path(ctypes.byref(shape))
 
 
 def bsa_attend_vs_workspace_bytes(shape: Shape, Wv: int, Ws: int) -> int:

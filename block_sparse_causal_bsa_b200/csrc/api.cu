@@ -63,15 +63,16 @@ bsa_status check_params(const bsa_shape* s, const bsa_select_params* p) {
   return BSA_OK;
 }
 
+bool attend_on_tensor_cores(const bsa_shape& s, int W) {
+  return bsa::attend_tc_supported(s) && W <= 1024 && (long long)s.B * s.Hq * s.N < (1ll << 31);
+}
+
 struct ScoreWs {
   float* kbar;       // pooled keys, or kmin (bounds)
   float* kbar2;      // kmax (bounds)
-  uint16_t* h16;     // fp16 pooled keys scaled by 2^r per block (mean kinds, tensor cores)
+  uint16_t* h16;     // fp16 tensor-core operand scaled by 2^r per block: pooled keys, or mid
+  uint16_t* h16b;    // bounds: rad, same scale
   float* kinv;       // 2^-r per block
-  uint16_t* hi;      // bounds, tensor cores: bf16 hi/lo of mid and rad
-  uint16_t* lo;
-  uint16_t* hi2;
-  uint16_t* lo2;
   float* w;          // value-block term (output-aware kinds)
   size_t bytes;
 };
@@ -91,14 +92,10 @@ ScoreWs score_ws(const bsa_shape& s, bsa_score_kind kind, void* base) {
   w.kbar = (float*)(p + off); off += align256(nk * s.d * 4);
   if (bounds) {
     w.kbar2 = (float*)(p + off); off += align256(nk * s.d * 4);
-    w.hi = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
-    w.lo = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
-    w.hi2 = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
-    w.lo2 = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
-  } else {
-    w.h16 = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
-    w.kinv = (float*)(p + off); off += align256(nk * 4);
+    w.h16b = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
   }
+  w.h16 = (uint16_t*)(p + off); off += align256(nk * s.d * 2);
+  w.kinv = (float*)(p + off); off += align256(nk * 4);
   if (vterm) {
     w.w = (float*)(p + off); off += align256(nk * 4);
   }
@@ -193,9 +190,9 @@ bsa_status run_score(const bsa_shape& s, bsa_score_kind kind, float beta, const 
   cudaError_t e;
   if (kind == BSA_SCORE_KMINMAX) {
     const bool tc = bsa::score_tc_supported(s);
-    e = bsa::launch_pool_bounds(s, k, w.kbar, w.kbar2, tc ? w.hi : nullptr, w.lo, w.hi2, w.lo2, cs);
+    e = bsa::launch_pool_bounds(s, k, w.kbar, w.kbar2, tc ? w.h16 : nullptr, w.h16b, w.kinv, cs);
     if (e != cudaSuccess) return cuda_fail(e, "pool (bounds)");
-    e = tc ? bsa::launch_score_tc_bounds(s, q, w.hi, w.lo, w.hi2, w.lo2, scores, dev_status, cs)
+    e = tc ? bsa::launch_score_tc_bounds(s, q, w.h16, w.h16b, w.kinv, scores, dev_status, cs)
            : bsa::launch_score_simt(s, q, w.kbar, w.kbar2, nullptr, 0, scores, cs);
     if (e != cudaSuccess) return cuda_fail(e, tc ? "score (tensor cores)" : "score");
     return BSA_OK;
@@ -393,8 +390,7 @@ bsa_status bsa_attend(const bsa_shape* s, const void* q, const void* k, const vo
   cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), cs);
   if (e != cudaSuccess) return cuda_fail(e, "clear dev_status");
   // tensor-core path for its shapes (bf16, d 128, blocks 64, tiles 128); CUDA cores otherwise
-  if (bsa::attend_tc_supported(*s) && W <= 1024 &&
-      (long long)s->B * s->Hq * s->N < (1ll << 31)) {
+  if (attend_on_tensor_cores(*s, W)) {
     e = bsa::launch_attend_tc(*s, q, k, v, kv_idx, kv_cnt, W, scale, out, lse, dev_status, cs);
     if (e != cudaSuccess) return cuda_fail(e, "attend (tensor cores)");
   } else {
@@ -536,6 +532,24 @@ bsa_status bsa_decode_list(const bsa_decode_shape* s, const bsa_decode_params* p
                          block_list, list_cnt, list_width);
   if (e != cudaSuccess) return cuda_fail(e, "decode_list");
   return ok();
+}
+
+// ---- which kernels a call runs ----------------------------------------------------------
+
+int bsa_attend_path(const bsa_shape* s, int W) {
+  if (check_shape(s) != BSA_OK || W < 1 || W > s->N / s->block_k) return -1;
+  return attend_on_tensor_cores(*s, W) ? BSA_PATH_TENSOR_CORES : BSA_PATH_CUDA_CORES;
+}
+
+int bsa_score_path(const bsa_shape* s, bsa_score_kind kind) {
+  if (check_shape(s) != BSA_OK || !known_kind(kind)) return -1;
+  const bool tc = kind == BSA_SCORE_KMINMAX ? bsa::score_tc_supported(*s) : bsa::score_rank_supported(*s);
+  return tc ? BSA_PATH_TENSOR_CORES : BSA_PATH_CUDA_CORES;
+}
+
+int bsa_decode_path(const bsa_decode_shape* s) {
+  if (!s || s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->L < 1 || s->Hq % s->Hkv) return -1;
+  return bsa::decode_tc_supported(*s) ? BSA_PATH_TENSOR_CORES : BSA_PATH_CUDA_CORES;
 }
 
 }  // extern "C"

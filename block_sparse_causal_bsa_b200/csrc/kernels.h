@@ -17,10 +17,10 @@ cudaError_t launch_pool(const bsa_shape& s, const void* k, const void* v, float*
                         int wlog = 0, float beta = 0.f);
 
 // Per-coordinate key bounds: kmin, kmax fp32 [B,Hkv,n_kb,d]; for the tensor-core score
-// (pointers may be null) the bf16 hi/lo splits of mid = (kmin+kmax)/2, rad = (kmax-kmin)/2.
+// (pointers may be null) mid = (kmin+kmax)/2 and rad = (kmax-kmin)/2 as fp16 scaled by
+// 2^r per block, and kinv [B,Hkv,n_kb] = 2^-r.
 cudaError_t launch_pool_bounds(const bsa_shape& s, const void* k, float* kmin, float* kmax,
-                               uint16_t* mid_hi, uint16_t* mid_lo, uint16_t* rad_hi, uint16_t* rad_lo,
-                               cudaStream_t st);
+                               uint16_t* mid16, uint16_t* rad16, float* kinv, cudaStream_t st);
 
 // Block scores on CUDA cores (fp32). kbar2 != null selects the bounds backbone (kbar =
 // kmin, kbar2 = kmax). wmode: 0 none, 1 times wnorm, 2 plus wnorm.
@@ -28,13 +28,12 @@ cudaError_t launch_score_simt(const bsa_shape& s, const void* q, const float* kb
                               const float* kbar2, const float* wnorm, int wmode, float* scores,
                               cudaStream_t st);
 
-// K-min/K-max block scores on tcgen05 tensor cores (bf16 inputs; mid and rad of the key
-// boxes as bf16 hi/lo pairs).
+// K-min/K-max block scores on tcgen05 tensor cores (bf16 inputs; mid16/rad16/kinv from
+// launch_pool_bounds).
 bool score_tc_supported(const bsa_shape& s);
-cudaError_t launch_score_tc_bounds(const bsa_shape& s, const void* q, const uint16_t* mid_hi,
-                                   const uint16_t* mid_lo, const uint16_t* rad_hi,
-                                   const uint16_t* rad_lo, float* scores, int32_t* dev_status,
-                                   cudaStream_t st);
+cudaError_t launch_score_tc_bounds(const bsa_shape& s, const void* q, const uint16_t* mid16,
+                                   const uint16_t* rad16, const float* kinv, float* scores,
+                                   int32_t* dev_status, cudaStream_t st);
 
 // Mean-pooled block scores on tcgen05 (fp16 operands with power-of-two scales), persistent,
 // optionally fused with the ranking of the selection. kbar16/kinv from launch_pool.

@@ -7,7 +7,8 @@
 // w = beta * max(0, ln ||Vbar_j||^2) (the additive form of [Stem] 2.B).
 // Bounds pool ([UGS] Metodologia step 1, the K-min/K-max backbone): per-coordinate
 // minimum and maximum of the block's keys, and for the tensor-core score the
-// box centre (kmin+kmax)/2 and half-width (kmax-kmin)/2 as bf16 hi/lo pairs.
+// box centre (kmin+kmax)/2 and half-width (kmax-kmin)/2 as fp16 with a per-block
+// power-of-two scale.
 //
 // Score ([UGS] step 2): s(t,j) = max over the tile's rows of q_i . Kbar_j
 // (times w_j, or plus w_j, for the output-aware forms), or of
@@ -115,19 +116,24 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ k, cons
 }
 
 // One CTA per (b, g, key block), 256 threads as in pool_kernel: per-coordinate
-// min and max over the block's keys (exact: they are input values).
+// min and max over the block's keys (exact: they are input values). With mid16 given,
+// also the box centre mid = (kmin+kmax)/2 and half-width rad = (kmax-kmin)/2 as fp16,
+// both scaled by one power of two 2^r per block (r chosen so that the block's largest
+// of |mid| and rad lands in [2^14, 2^15)), and kinv[block] = 2^-r: the operands of the
+// tensor-core bounds score, where max(q a, q b) = q (a+b)/2 + |q| (b-a)/2 for b >= a.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) pool_bounds_kernel(const T* __restrict__ k, int N, int block_k,
                                                           float* __restrict__ kmin,
                                                           float* __restrict__ kmax,
-                                                          uint16_t* __restrict__ mid_hi,
-                                                          uint16_t* __restrict__ mid_lo,
-                                                          uint16_t* __restrict__ rad_hi,
-                                                          uint16_t* __restrict__ rad_lo) {
+                                                          uint16_t* __restrict__ mid16,
+                                                          uint16_t* __restrict__ rad16,
+                                                          float* __restrict__ kinv) {
   constexpr int CPT = 8;
   constexpr int TPR = D / CPT;
   constexpr int PHASES = 256 / TPR;
   __shared__ float rmin[PHASES][D], rmax[PHASES][D];
+  __shared__ float smid[D], srad[D];
+  __shared__ int rexp;
   const int j = blockIdx.x;
   const size_t bg = blockIdx.y;
   const int n_kb = N / block_k;
@@ -155,15 +161,34 @@ __global__ void __launch_bounds__(256) pool_bounds_kernel(const T* __restrict__ 
     const size_t o = (bg * n_kb + j) * D + c;
     kmin[o] = a;
     kmax[o] = b;
-    if (mid_hi) {
-      // max(q a, q b) = q (a+b)/2 + |q| (b-a)/2 for b >= a
-      const float mid = 0.5f * (a + b), rad = 0.5f * (b - a);
-      const uint16_t mh = f32_to_bf16_rn(mid), rh = f32_to_bf16_rn(rad);
-      mid_hi[o] = mh;
-      mid_lo[o] = f32_to_bf16_rn(mid - bf16_to_f32(mh));
-      rad_hi[o] = rh;
-      rad_lo[o] = f32_to_bf16_rn(rad - bf16_to_f32(rh));
+    smid[c] = 0.5f * (a + b);
+    srad[c] = 0.5f * (b - a);
+  }
+  if (!mid16) return;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float mx = 0.f;
+    for (int c = threadIdx.x; c < D; c += 32) mx = fmaxf(mx, fmaxf(fabsf(smid[c]), srad[c]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (threadIdx.x == 0) {
+      const uint32_t u = __float_as_uint(mx);
+      int r = 0;
+      if (u != 0u && u < 0x7f800000u) {
+        r = 14 - ((int)(u >> 23) - 127);
+        r = r < -126 ? -126 : (r > 126 ? 126 : r);
+      }
+      rexp = r;
+      kinv[bg * n_kb + j] = __int_as_float((127 - r) << 23);
     }
+  }
+  __syncthreads();
+  const float sc = __int_as_float((127 + rexp) << 23);
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    const size_t o = (bg * n_kb + j) * D + c;
+    const __half m = __float2half_rn(smid[c] * sc), r = __float2half_rn(srad[c] * sc);
+    mid16[o] = *reinterpret_cast<const uint16_t*>(&m);
+    rad16[o] = *reinterpret_cast<const uint16_t*>(&r);
   }
 }
 
@@ -194,12 +219,11 @@ cudaError_t launch_pool(const bsa_shape& s, const void* k, const void* v, float*
 }
 
 cudaError_t launch_pool_bounds(const bsa_shape& s, const void* k, float* kmin, float* kmax,
-                               uint16_t* mid_hi, uint16_t* mid_lo, uint16_t* rad_hi, uint16_t* rad_lo,
-                               cudaStream_t st) {
+                               uint16_t* mid16, uint16_t* rad16, float* kinv, cudaStream_t st) {
   dim3 grid(s.N / s.block_k, s.B * s.Hkv);
 #define BSA_POOLB(T, D)                                                                            \
-  pool_bounds_kernel<T, D><<<grid, 256, 0, st>>>((const T*)k, s.N, s.block_k, kmin, kmax, mid_hi, \
-                                                 mid_lo, rad_hi, rad_lo)
+  pool_bounds_kernel<T, D><<<grid, 256, 0, st>>>((const T*)k, s.N, s.block_k, kmin, kmax, mid16, \
+                                                 rad16, kinv)
   if (s.dtype == BSA_BF16) {
     if (s.d == 128) BSA_POOLB(uint16_t, 128); else BSA_POOLB(uint16_t, 64);
   } else {

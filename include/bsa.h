@@ -38,7 +38,8 @@
  *              the call clears *dev_status first, the offending work is
  *              skipped, and the kernel never traps.
  *   Precision  bf16 inputs, fp32 accumulation and softmax; BSA_F32 inputs run
- *              an fp32 CUDA-core path.
+ *              an fp32 CUDA-core path, and so do a few bf16 shapes (see the
+ *              bsa_*_path queries below, which report the choice).
  */
 #ifndef BSA_H
 #define BSA_H
@@ -349,6 +350,27 @@ bsa_status bsa_select_noalloc(const bsa_shape* shape, const bsa_select_params* p
  * context stays usable afterwards. Returns BSA_ERR_INVALID_ARG for another mode or a
  * null pointer, BSA_ERR_CUDA if the launch fails. */
 bsa_status bsa_selftest_wait(int mode, int32_t* dev_status, int32_t* completed, void* stream);
+
+/* ---- which kernels a call runs ------------------------------------------------------ */
+
+/* The compute calls pick their kernels from the shape alone. These queries return the
+ * choice without launching anything: BSA_PATH_TENSOR_CORES (tcgen05/TMEM/TMA kernels),
+ * BSA_PATH_CUDA_CORES (fp32 CUDA-core kernels, about an order of magnitude slower on
+ * large problems), or -1 for arguments the call itself would reject.
+ *   bsa_score_path   tensor cores for bf16 inputs with d = 128 and query tiles of 128
+ *                    (any key block); CUDA cores for BSA_F32 inputs, d = 64 or query tiles
+ *                    of 64. The same holds for bsa_score_select, which ranks inside the
+ *                    tensor-core score kernel for the mean-pooled kinds.
+ *   bsa_attend_path  tensor cores for bf16, d = 128, key blocks of 64, query tiles of 128,
+ *                    W <= 1024 and B*Hq*N < 2^31; CUDA cores for every other shape
+ *                    (BSA_F32, d = 64, key blocks of 128, query tiles of 64, W > 1024).
+ *   bsa_decode_path  tensor cores for d = 128, block_kv = 128, Hq/Hkv <= 8 and
+ *                    B*Hkv*L < 2^31; CUDA cores for d = 64 or block_kv = 64.
+ * bsa_attend_vs always runs on tensor cores (other shapes are rejected). */
+enum { BSA_PATH_CUDA_CORES = 0, BSA_PATH_TENSOR_CORES = 1 };
+int bsa_score_path(const bsa_shape* shape, bsa_score_kind kind);
+int bsa_attend_path(const bsa_shape* shape, int W);
+int bsa_decode_path(const bsa_decode_shape* shape);
 
 /* ---- misc --------------------------------------------------------------------------- */
 

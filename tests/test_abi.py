@@ -141,7 +141,7 @@ def test_score_kinds_validation():
     nkb = 8 * 2048
     n_mean = bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_MEAN)
     assert bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_MEAN_VLOG) >= n_mean + nkb * 4
-    assert bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_KMINMAX) >= 2 * n_mean
+    assert bb.bsa_score_workspace_bytes(s, bb.BSA_SCORE_KMINMAX) >= n_mean + nkb * 128 * (4 + 2)   # + kmax, rad
     assert bb.bsa_score_workspace_bytes(s, 7) == 0
     big = 1 << 34
     # the additive form needs beta: not through bsa_score, not with NULL params
@@ -256,3 +256,35 @@ def test_decode_cache_too_large_rejected():
     assert L.bsa_decode(ctypes.byref(ds), ctypes.byref(dp), 16, 16, 16, 0.1, 16, 16, None, 16,
                         None) == bb.BSA_ERR_UNSUPPORTED
     assert b"2^31" in L.bsa_last_error()
+
+
+def test_kernel_path_queries():
+    """Every shape the header lists as a CUDA-core fallback reports it, the workloads' shapes
+    report tensor cores, and invalid arguments report -1 (nothing is launched)."""
+    TC, CC = bb.BSA_PATH_TENSOR_CORES, bb.BSA_PATH_CUDA_CORES
+    base = dict(B=1, Hq=32, Hkv=8, N=131072, d=128, block_k=64, tile_q=128, dtype=bb.BSA_BF16)
+
+    def sh(**kw):
+        a = dict(base, **kw)
+        return bb.Shape(a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["block_k"], a["tile_q"], a["dtype"])
+    # attend
+    assert bb.bsa_attend_path(sh(), 128) == TC
+    assert bb.bsa_attend_path(sh(), 1024) == TC
+    assert bb.bsa_attend_path(sh(), 1025) == CC
+    for kw in (dict(dtype=bb.BSA_F32), dict(d=64), dict(block_k=128), dict(tile_q=64)):
+        assert bb.bsa_attend_path(sh(**kw), 64) == CC, kw
+    assert bb.bsa_attend_path(sh(B=256, Hq=64, Hkv=8), 64) == CC         # B*Hq*N = 2^31
+    assert bb.bsa_attend_path(sh(), 0) == -1 and bb.bsa_attend_path(sh(d=96), 64) == -1
+    # score (and the fused score+select)
+    for kind in range(4):
+        assert bb.bsa_score_path(sh(), kind) == TC
+        assert bb.bsa_score_path(sh(block_k=128), kind) == TC
+        for kw in (dict(dtype=bb.BSA_F32), dict(d=64), dict(tile_q=64)):
+            assert bb.bsa_score_path(sh(**kw), kind) == CC, (kind, kw)
+    assert bb.bsa_score_path(sh(), 9) == -1
+    # decode
+    assert bb.bsa_decode_path(bb.DecodeShape(16, 32, 8, 65536, 128, 128, bb.BSA_BF16)) == TC
+    assert bb.bsa_decode_path(bb.DecodeShape(2, 8, 8, 4096, 128, 128, bb.BSA_BF16)) == TC
+    assert bb.bsa_decode_path(bb.DecodeShape(2, 8, 2, 4096, 64, 128, bb.BSA_BF16)) == CC
+    assert bb.bsa_decode_path(bb.DecodeShape(2, 8, 2, 4096, 128, 64, bb.BSA_BF16)) == CC
+    assert bb.bsa_decode_path(bb.DecodeShape(2, 6, 4, 4096, 128, 128, bb.BSA_BF16)) == -1
