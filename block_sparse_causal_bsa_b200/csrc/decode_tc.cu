@@ -59,7 +59,7 @@ constexpr uint32_t kTmemCols = 64;        // S[2] at 0/16, D[2] at 32/48
 struct __align__(8) Ctrl {
   uint64_t kv_full[STAGES], kv_empty[STAGES];
   uint64_t s_full[2], o_full[2];
-  uint64_t red_max, p_ready[2], probe_rdy, decided, done, vote;
+  uint64_t p_ready[2], probe_rdy, decided, done, vote;
   uint32_t tmem;
   int abort_flag;     // error: softmax warps unwind
   int halt;           // producer / MMA stop issuing (normal stop or error)
@@ -68,7 +68,7 @@ struct __align__(8) Ctrl {
   float lpart[2][4];            // [block parity][warp] row-sum part of the first head
   float xfull[2][HD];           // [block parity][head dim] unnormalised O of the first head
   float lfin[4][GMAX];          // [warp][head] final row-sum parts
-  double prod[3][kMaxProbe];   // decider: per-coordinate fp64 products of the current block
+  double prod[2][kMaxProbe];   // decider: per-coordinate fp64 products of the current block
   int swait[2][4];              // softmax warps' wait results for S_t, by t parity
   int n_steps;                  // blocks to visit
   uint16_t blk[kMaxDecodeList]; // visit list (decode over a block list)
@@ -96,6 +96,7 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col, uint32_t half_by
 }
 }  // namespace
 
+template <int G>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
     const uint16_t* __restrict__ q, const DecodeArgs a, uint16_t* __restrict__ out,
@@ -106,7 +107,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bg = blockIdx.x;
   const int b = bg / a.Hkv, g = bg % a.Hkv;
-  const int G = a.Hq / a.Hkv;
   const int nb = a.L / BKV;
   const int row0 = bg * a.L;
   const uint32_t sStages = tc::smem_u32(sm + kSmemStages);
@@ -122,7 +122,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       tc::mbar_init(&c.s_full[i], 1);
       tc::mbar_init(&c.o_full[i], 1);
     }
-    tc::mbar_init(&c.red_max, 4);
     tc::mbar_init(&c.vote, 4);
     tc::mbar_init(&c.p_ready[0], 4);
     tc::mbar_init(&c.p_ready[1], 4);
@@ -170,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   volatile int* halt = &c.halt;
   int issued = 0;
   bool mma_issued = false;
-  float o_fin[GMAX];        // softmax warps: unnormalised output of this thread's head dim
+  float o_fin[G];           // softmax warps: unnormalised output of this thread's head dim
   bool out_ok = false;
 
   if (warp == 0 && lane == 0) {
@@ -233,73 +232,69 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;           // key of S_t, head dim of D_t
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    float m[GMAX], lw[GMAX], o[GMAX];
+    // m, o per head; lw[0] is this warp's part of the first head's row sum (the probe needs
+    // it after every block), lw[h > 0] this thread's part (reduced once, at the end)
+    float m[G], lw[G], o[G];
 #pragma unroll
-    for (int h = 0; h < GMAX; ++h) { m[h] = -INFINITY; lw[h] = 0.f; o[h] = 0.f; }
-    // softmax of block t: writes P_t, returns alpha_t and this warp's part of the block sums.
-    // 0: done; 1: a stop was decided before S_t arrived (the MMA issuer may never issue it:
-    // it halts once the decider stops, possibly before block t landed); 2: error.
-    auto softmax = [&](int t, float (&alpha)[GMAX], float (&ps)[GMAX]) -> int {
+    for (int h = 0; h < G; ++h) { m[h] = -INFINITY; lw[h] = 0.f; o[h] = 0.f; }
+    // softmax of block t: writes P_t, returns alpha_t and the block sums (ps[0]: this warp's
+    // part; ps[h > 0]: this thread's key). 0: done; 1: a stop was decided before S_t arrived
+    // (the MMA issuer may never issue it: it halts once the decider stops, possibly before
+    // block t landed); 2: error.
+    auto softmax = [&](int t, float (&alpha)[G], float (&ps)[G]) -> int {
       const int buf = t & 1;
       const int w = __reduce_max_sync(0xffffffffu, (unsigned)tc::mbar_wait_or_halt(
                                           &c.s_full[buf], (t >> 1) & 1, halt, abort_flag, dev_status));
-      // the four warps act on one verdict (one may see S_t land while another sees the halt
-      // first): each posts its result and arrives on `vote` (phase t); a warp writes slot
-      // t&1 again only after every warp arrived for t+1, i.e. read its slot-t verdicts
+      float sc[G];
+      if (w == 0) {
+        // S_t landed for this warp: its scores and, per head, the warp's block max as an
+        // order-preserving key reduced in one instruction
+        tc::tc_fence_after();
+        uint32_t sv[16];
+        tc::tmem_ld16(tl + buf * NPAD, sv);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          sc[h] = __uint_as_float(sv[h]);
+          const uint32_t key = (sv[h] & 0x80000000u) ? ~sv[h] : (sv[h] | 0x80000000u);
+          const uint32_t mk = __reduce_max_sync(0xffffffffu, key);
+          if (lane == 0) c.rmax[buf][quarter][h] = __uint_as_float((mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk);
+        }
+      }
+      // one handshake for both: the four warps act on one verdict (one may see S_t land while
+      // another sees the halt first) and exchange their block maxima. Each posts its result
+      // (and maxima) and arrives on `vote` (phase t); a warp writes slot t&1 again only after
+      // every warp arrived for t+1, i.e. read its slot-t values
       if (lane == 0) c.swait[t & 1][quarter] = w;
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c.vote);
       if (!warp_all(tc::mbar_wait(&c.vote, t & 1, abort_flag, dev_status))) return 2;
       const int v = max(max(c.swait[t & 1][0], c.swait[t & 1][1]), max(c.swait[t & 1][2], c.swait[t & 1][3]));
       if (v != 0) return v;
-      tc::tc_fence_after();
-      uint32_t sv[16];
-      tc::tmem_ld16(tl + buf * NPAD, sv);
-      float sc[GMAX];
-#pragma unroll
-      for (int h = 0; h < GMAX; ++h) {
-        float v = h < G ? __uint_as_float(sv[h]) : -INFINITY;
-        sc[h] = v;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-        if (lane == 0 && h < G) c.rmax[buf][quarter][h] = v;
-      }
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&c.red_max);
-      if (!warp_all(tc::mbar_wait(&c.red_max, t & 1, abort_flag, dev_status))) return 2;
       uint8_t* pbase = sm + kSmemP + buf * 2 * kSmallHalf;
 #pragma unroll
-      for (int h = 0; h < GMAX; ++h) {
-        if (h < G) {
-          const float bmax = fmaxf(fmaxf(c.rmax[buf][0][h], c.rmax[buf][1][h]),
-                                   fmaxf(c.rmax[buf][2][h], c.rmax[buf][3][h]));
-          const float mn = fmaxf(m[h], bmax * a.scale_log2);
-          alpha[h] = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mn);
-          m[h] = mn;
-          const float p = ex2(fmaf(sc[h], a.scale_log2, -mn));
-          *reinterpret_cast<__nv_bfloat16*>(pbase + sw128_off(h, r, kSmallHalf)) = __float2bfloat16_rn(p);
-          ps[h] = p;
-        } else {
-          alpha[h] = 1.f;
-          ps[h] = 0.f;
-        }
+      for (int h = 0; h < G; ++h) {
+        const float bmax = fmaxf(fmaxf(c.rmax[buf][0][h], c.rmax[buf][1][h]),
+                                 fmaxf(c.rmax[buf][2][h], c.rmax[buf][3][h]));
+        const float mn = fmaxf(m[h], bmax * a.scale_log2);
+        alpha[h] = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mn);
+        m[h] = mn;
+        const float p = ex2(fmaf(sc[h], a.scale_log2, -mn));
+        *reinterpret_cast<__nv_bfloat16*>(pbase + sw128_off(h, r, kSmallHalf)) = __float2bfloat16_rn(p);
+        ps[h] = p;
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c.p_ready[buf]);     // the MMA issuer may start PV_t
+      float v0 = ps[0];
 #pragma unroll
-      for (int h = 0; h < GMAX; ++h) {
-        float v = ps[h];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        ps[h] = v;
-      }
+      for (int off = 16; off > 0; off >>= 1) v0 += __shfl_xor_sync(0xffffffffu, v0, off);
+      ps[0] = v0;
       return 0;
     };
     int used = ns;
     bool ok = true;
-    float a_cur[GMAX], p_cur[GMAX], a_nxt[GMAX], p_nxt[GMAX];
+    float a_cur[G], p_cur[G], a_nxt[G], p_nxt[G];
     if (ns > 0) ok = softmax(0, a_cur, p_cur) == 0;  // an empty visit list leaves O = 0
     for (int t = 0; ok && t < ns; ++t) {
       const int buf = t & 1;
@@ -332,11 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         }
       }
 #pragma unroll
-      for (int h = 0; h < GMAX; ++h) {
-        if (h < G) {
-          o[h] = fmaf(o[h], a_cur[h], __uint_as_float(dv[h]));
-          lw[h] = fmaf(lw[h], a_cur[h], p_cur[h]);
-        }
+      for (int h = 0; h < G; ++h) {
+        o[h] = fmaf(o[h], a_cur[h], __uint_as_float(dv[h]));
+        lw[h] = fmaf(lw[h], a_cur[h], p_cur[h]);
         a_cur[h] = a_nxt[h];
         p_cur[h] = p_nxt[h];
       }
@@ -345,9 +338,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&c.probe_rdy);
     }
+#pragma unroll
+    for (int h = 1; h < G; ++h) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) lw[h] += __shfl_xor_sync(0xffffffffu, lw[h], off);
+    }
     if (lane == 0) {
 #pragma unroll
-      for (int h = 0; h < GMAX; ++h) c.lfin[quarter][h] = lw[h];
+      for (int h = 0; h < G; ++h) c.lfin[quarter][h] = lw[h];
     }
     if (threadIdx.x == 64) {
       *halt = 1;                       // nothing more to stream
@@ -356,17 +354,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     // the output is written after the teardown barrier, when every warp's l part is in
     out_ok = warp_all(ok);
 #pragma unroll
-    for (int h = 0; h < GMAX; ++h) o_fin[h] = o[h];
+    for (int h = 0; h < G; ++h) o_fin[h] = o[h];
   } else if (warp == 6) {
     // ---------------- decider ----------------
     // Lane i owns probe coordinates i and i + 32: it forms x = O / l for them (the
     // fp32 divisions run in parallel), writes the trace, and the exact fp64 products
-    // x_t^2, x_{t-1}^2, x_t x_{t-1} (products of fp32 values are exact in fp64).
-    // Lane 0 adds them up in coordinate order, then tests stability.
+    // x_t^2 and x_t x_{t-1} (products of fp32 values are exact in fp64). Lane 0 adds
+    // them up in coordinate order, then tests stability; ||x_{t-1}||^2 and its root are
+    // the previous block's, the same sum in the same order.
     const int np = a.n_probe;
     const int d0 = lane < np ? a.dims[lane] : 0;
     const int d1 = lane + 32 < np ? a.dims[lane + 32] : 0;
     float xp0 = 0.f, xp1 = 0.f;
+    double np_prev = 0.0;          // lane 0: ||x_{t-1}||
     int run = 0;
     for (int t = 0; t < ns; ++t) {
       if (!warp_all(tc::mbar_wait(&c.probe_rdy, t & 1, abort_flag, dev_status))) break;
@@ -380,24 +380,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         if (lane + 32 < np) tr[lane + 32] = x1;
       }
       c.prod[0][lane] = __dmul_rn((double)x0, (double)x0);
-      c.prod[1][lane] = __dmul_rn((double)xp0, (double)xp0);
-      c.prod[2][lane] = __dmul_rn((double)x0, (double)xp0);
+      c.prod[1][lane] = __dmul_rn((double)x0, (double)xp0);
       c.prod[0][lane + 32] = __dmul_rn((double)x1, (double)x1);
-      c.prod[1][lane + 32] = __dmul_rn((double)xp1, (double)xp1);
-      c.prod[2][lane + 32] = __dmul_rn((double)x1, (double)xp1);
+      c.prod[1][lane + 32] = __dmul_rn((double)x1, (double)xp1);
       xp0 = x0;
       xp1 = x1;
       __syncwarp();
       if (lane == 0) {
         bool stop = false;
+        double sc2 = 0.0, dt = 0.0;
         if (t >= 1) {
-          double sc2 = 0.0, sp2 = 0.0, dt = 0.0;
           for (int i = 0; i < np; ++i) {
             sc2 = __dadd_rn(sc2, c.prod[0][i]);
-            sp2 = __dadd_rn(sp2, c.prod[1][i]);
-            dt = __dadd_rn(dt, c.prod[2][i]);
+            dt = __dadd_rn(dt, c.prod[1][i]);
           }
-          const double nc = __dsqrt_rn(sc2), npv = __dsqrt_rn(sp2);
+        } else {
+          for (int i = 0; i < np; ++i) sc2 = __dadd_rn(sc2, c.prod[0][i]);
+        }
+        const double nc = __dsqrt_rn(sc2), npv = np_prev;
+        np_prev = nc;
+        if (t >= 1) {
           const double ds = fabs(__dadd_rn(nc, -npv));
           const double den = __dmul_rn(nc, npv);
           const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
@@ -436,18 +438,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     const int r = (warp & 3) * 32 + lane;
     uint16_t* og = out + ((size_t)b * a.Hq + (size_t)g * G) * HD;
 #pragma unroll
-    for (int h = 0; h < GMAX; ++h) {
-      if (h < G) {
-        const float lt = (c.lfin[0][h] + c.lfin[1][h]) + (c.lfin[2][h] + c.lfin[3][h]);
-        og[h * HD + r] = f32_to_bf16_rn(lt > 0.f ? o_fin[h] / lt : 0.f);
-      }
+    for (int h = 0; h < G; ++h) {
+      const float lt = (c.lfin[0][h] + c.lfin[1][h]) + (c.lfin[2][h] + c.lfin[3][h]);
+      og[h * HD + r] = f32_to_bf16_rn(lt > 0.f ? o_fin[h] / lt : 0.f);
     }
   }
 }
 
 bool decode_tc_supported(const bsa_decode_shape& s) {
   const int G = s.Hq / s.Hkv;
-  return s.dtype == BSA_BF16 && s.d == HD && s.block_kv == BKV && G >= 1 && G <= GMAX &&
+  return s.dtype == BSA_BF16 && s.d == HD && s.block_kv == BKV && (G == 1 || G == 2 || G == 4 || G == 8) &&
          (long long)s.B * s.Hkv * s.L < (1ll << 31);
 }
 
@@ -458,12 +458,18 @@ cudaError_t launch_decode_tc(const bsa_decode_shape& s, const DecodeArgs& a, con
   const uint64_t rows = (uint64_t)s.B * s.Hkv * s.L;
   if (!make_tmap_bf16_2d(&mk, kc, rows, HD, 64, BKV) || !make_tmap_bf16_2d(&mv, vc, rows, HD, 64, BKV))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+  auto kern = decode_tc_kernel<1>;
+  switch (s.Hq / s.Hkv) {
+    case 1: kern = decode_tc_kernel<1>; break;
+    case 2: kern = decode_tc_kernel<2>; break;
+    case 4: kern = decode_tc_kernel<4>; break;
+    case 8: kern = decode_tc_kernel<8>; break;
+    default: return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<<<s.B * s.Hkv, kThreads, kSmemBytes, st>>>(mk, mv, (const uint16_t*)q, a,
-                                                             (uint16_t*)out, blocks_used, probe_trace,
-                                                             dev_status);
+  kern<<<s.B * s.Hkv, kThreads, kSmemBytes, st>>>(mk, mv, (const uint16_t*)q, a, (uint16_t*)out, blocks_used,
+                                                  probe_trace, dev_status);
   return cudaGetLastError();
 }
 
