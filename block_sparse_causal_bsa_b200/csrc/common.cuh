@@ -119,6 +119,16 @@ __device__ inline int warp_compact_blocks(const int32_t* lst, int cnt, int cap, 
   return n;
 }
 
+// Sum over a warp of fp64 terms in the order the [ART] 2.2 probe sums take here: each
+// lane passes the rounded sum of its two terms (probe coordinates lane and lane + 32, zero
+// where there is none); the values 16, 8, 4, 2 and 1 lanes apart are then added, each add
+// rounded. Every lane returns the same sum (fp64 addition is commutative).
+__device__ __forceinline__ double warp_pairwise_sum(double v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
 // Order-preserving map of an fp32 score to uint32 (larger score -> larger key).
 // -0.0 is folded into +0.0 so that equal scores compare equal, as IEEE does.
 __device__ __forceinline__ uint32_t score_key(float s) {

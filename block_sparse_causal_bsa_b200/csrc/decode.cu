@@ -8,8 +8,9 @@
 // After every block it forms the probe x^(t) = O^(t)[first head][probe_dims]
 // (fp32, normalised) and, from block 1 on, tests stability in fp64:
 //   d_scale = | ||x_t|| - ||x_{t-1}|| |,  d_dir = 1 - x_t.x_{t-1} / (||x_t|| ||x_{t-1}||)
-// (d_dir = 1 when a norm is 0), sums in index order with separate multiply and
-// add ([ART] 2.2). A block is stable iff d_scale < tau and d_dir < phi; the
+// (d_dir = 1 when a norm is 0), exact products, and each sum over the probe
+// coordinates taken by warp 0 in the fixed pairwise order of warp_pairwise_sum
+// ([ART] 2.2). A block is stable iff d_scale < tau and d_dir < phi; the
 // stream stops after `patience` consecutive stable blocks ([ART] 2.3). Block 0
 // is always processed, because no test exists before block 1 ([ART] 2.4).
 //
@@ -202,24 +203,28 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
       if (probe_trace) probe_trace[((size_t)bg * tstride + blk) * a.n_probe + tid] = x;
     }
     __syncthreads();
-    if (tid == 0) {
+    if (tid < 32) {
+      // lane i: coordinates i and i + 32 (zero where there is none)
+      const int n = a.n_probe;
+      const double a0 = tid < n ? (double)xcur[tid] : 0.0, a1 = tid + 32 < n ? (double)xcur[tid + 32] : 0.0;
+      const double b0 = tid < n ? (double)xprev[tid] : 0.0, b1 = tid + 32 < n ? (double)xprev[tid + 32] : 0.0;
       if (blk >= 1) {
-        double sc = 0.0, sp = 0.0, dt = 0.0;
-        for (int i = 0; i < a.n_probe; ++i) {
-          const double xa = (double)xcur[i], xb = (double)xprev[i];
-          sc = __dadd_rn(sc, __dmul_rn(xa, xa));
-          sp = __dadd_rn(sp, __dmul_rn(xb, xb));
-          dt = __dadd_rn(dt, __dmul_rn(xa, xb));
+        const double sc = warp_pairwise_sum(__dadd_rn(__dmul_rn(a0, a0), __dmul_rn(a1, a1)));
+        const double sp = warp_pairwise_sum(__dadd_rn(__dmul_rn(b0, b0), __dmul_rn(b1, b1)));
+        const double dt = warp_pairwise_sum(__dadd_rn(__dmul_rn(a0, b0), __dmul_rn(a1, b1)));
+        if (tid == 0) {
+          const double nc = __dsqrt_rn(sc), np = __dsqrt_rn(sp);
+          const double ds = fabs(__dadd_rn(nc, -np));
+          const double den = __dmul_rn(nc, np);
+          const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
+          const bool stable = (ds < (double)a.tau) && (dd < (double)a.phi);
+          run_s = stable ? run_s + 1 : 0;
+          if (a.enable && run_s >= a.patience) stop_s = 1;
         }
-        const double nc = __dsqrt_rn(sc), np = __dsqrt_rn(sp);
-        const double ds = fabs(__dadd_rn(nc, -np));
-        const double den = __dmul_rn(nc, np);
-        const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
-        const bool stable = (ds < (double)a.tau) && (dd < (double)a.phi);
-        run_s = stable ? run_s + 1 : 0;
-        if (a.enable && run_s >= a.patience) stop_s = 1;
       }
-      for (int i = 0; i < a.n_probe; ++i) xprev[i] = xcur[i];
+      __syncwarp();
+      if (tid < n) xprev[tid] = xcur[tid];
+      if (tid + 32 < n) xprev[tid + 32] = xcur[tid + 32];
     }
     __syncthreads();
     if (stop_s) { used = blk + 1; break; }

@@ -19,21 +19,24 @@
 //                        handshake), P_t to shared memory (bf16, 128-byte swizzle),
 //                        then O[h][r] = O[h][r] * alpha_h + D_t[r][h] in registers;
 //                        each warp keeps its own part of the row sums l.
-//   warp 6 (one thread)  decider: for block t it forms the probe
+//   warp 6               decider: for block t it forms the probe
 //                        x^(t) = O^(t)[first head][probe dims] / l (fp32; l = the
 //                        four warp parts added in a fixed order) and runs the fp64
-//                        stability test (sums in index order, separate multiply and
-//                        add), then publishes stop / continue.
+//                        stability test (exact products, sums in a fixed pairwise
+//                        order across the warp), then publishes stop / continue.
 // The work is software-pipelined: the MMA issuer computes S_{t+1} before PV_t,
 // and the softmax warps produce P_{t+1} (two P buffers) before they fold D_t, so
 // the softmax of one block overlaps the value product of the previous one. The
-// decider judges block t while the softmax warps go on; they look at that
-// verdict only before folding D_{t+1}, and on a stop return the unfolded O^(t).
-// After a stop the producer and MMA threads are released through a halt flag;
-// the MMA issuer may then never issue S_{t+2}, so the softmax warps' wait for it
-// also watches the halt flag, and the four warps act on one verdict (posted per
-// warp and joined through the bounded `vote` mbarrier). The CTA then waits for
-// its own copies and MMAs and frees TMEM. All waits are bounded.
+// decider judges block t while the softmax warps go on with blocks t+1 and t+2;
+// they read that verdict only before folding D_{t+2}, keeping a copy of O^(t)
+// until then, and on a stop return that copy. After a stop the producer and MMA
+// threads are released through a halt flag; the MMA issuer may then never issue
+// the next S, so the softmax warps' wait for it also watches the halt flag (and
+// then reads the verdicts still open), and the four warps act on one verdict
+// (posted per warp and joined through the bounded `vote` mbarrier). The MMA
+// issuer keeps issuing PV_t for every P_t published until the softmax warps
+// leave. The CTA then waits for its own copies and MMAs and frees TMEM. All
+// waits are bounded.
 // Shapes: bf16, d = 128, KV blocks of 128, Hq/Hkv <= 8.
 #include <math.h>
 
@@ -59,16 +62,16 @@ constexpr uint32_t kTmemCols = 64;        // S[2] at 0/16, D[2] at 32/48
 struct __align__(8) Ctrl {
   uint64_t kv_full[STAGES], kv_empty[STAGES];
   uint64_t s_full[2], o_full[2];
-  uint64_t p_ready[2], probe_rdy, decided, done, vote;
+  uint64_t p_ready[2], probe_rdy[2], decided[2], done, vote;   // probe_rdy, decided: by block parity
   uint32_t tmem;
   int abort_flag;     // error: softmax warps unwind
   int halt;           // producer / MMA stop issuing (normal stop or error)
+  int sm_quit;        // the softmax warps left their loop: no further P_t will come
   int stop_at;        // block after which the decider stopped, or -1
   float rmax[2][4][GMAX];       // [block parity][warp][head]
   float lpart[2][4];            // [block parity][warp] row-sum part of the first head
   float xfull[2][HD];           // [block parity][head dim] unnormalised O of the first head
   float lfin[4][GMAX];          // [warp][head] final row-sum parts
-  double prod[2][kMaxProbe];   // decider: per-coordinate fp64 products of the current block
   int swait[2][4];              // softmax warps' wait results for S_t, by t parity
   int n_steps;                  // blocks to visit
   uint16_t blk[kMaxDecodeList]; // visit list (decode over a block list)
@@ -125,11 +128,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     tc::mbar_init(&c.vote, 4);
     tc::mbar_init(&c.p_ready[0], 4);
     tc::mbar_init(&c.p_ready[1], 4);
-    tc::mbar_init(&c.probe_rdy, 4);
-    tc::mbar_init(&c.decided, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&c.probe_rdy[i], 4);
+      tc::mbar_init(&c.decided[i], 1);
+    }
     tc::mbar_init(&c.done, 1);
     c.abort_flag = 0;
     c.halt = 0;
+    c.sm_quit = 0;
     c.stop_at = -1;
     tc::fence_mbar_init();
   }
@@ -167,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   const int tstride = a.blist ? a.list_w : nb;      // probe-trace rows per group
   volatile int* abort_flag = &c.abort_flag;
   volatile int* halt = &c.halt;
+  volatile int* sm_quit = &c.sm_quit;
   int issued = 0;
   bool mma_issued = false;
   float o_fin[G];           // softmax warps: unnormalised output of this thread's head dim
@@ -213,7 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     for (int t = 0; ok && t < ns; ++t) {
       // S_{t+1} first: its buffer held S_{t-1}, which the softmax warps read before P_{t-1}
       if (t + 1 < ns && !issue_s(t + 1)) break;
-      if (!tc::mbar_wait_halt(&c.p_ready[t & 1], (t >> 1) & 1, halt, dev_status)) break;
+      // P_t comes unless the softmax warps quit first (they do after a stop is seen or on
+      // an error); a halt alone must not skip PV_t once S_{t+1} is issued, since the
+      // softmax warps that received S_{t+1} then wait for D_t
+      if (!tc::mbar_wait_halt(&c.p_ready[t & 1], (t >> 1) & 1, sm_quit, dev_status)) break;
       tc::tc_fence_after();
       const int s = t % STAGES;
       const uint32_t vb = sStages + s * kStage + kTile;
@@ -240,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     // softmax of block t: writes P_t, returns alpha_t and the block sums (ps[0]: this warp's
     // part; ps[h > 0]: this thread's key). 0: done; 1: a stop was decided before S_t arrived
     // (the MMA issuer may never issue it: it halts once the decider stops, possibly before
-    // block t landed); 2: error.
+    // block t landed); 2: error. P_t is published (p_ready) only when 0 is returned.
     auto softmax = [&](int t, float (&alpha)[G], float (&ps)[G]) -> int {
       const int buf = t & 1;
       const int w = __reduce_max_sync(0xffffffffu, (unsigned)tc::mbar_wait_or_halt(
@@ -295,39 +305,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
     int used = ns;
     bool ok = true;
     float a_cur[G], p_cur[G], a_nxt[G], p_nxt[G];
+    // O^(t-2) and its row-sum parts: the verdict on a block is read two blocks later, so
+    // the decider's test runs beside the next block's softmax and fold
+    float o_sv[G], l_sv[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) { o_sv[h] = 0.f; l_sv[h] = 0.f; }
+    // after a halt seen in block t: the stop is on block t-2 or t-1 (the verdicts before
+    // were read, and said go on). Returns that block, or -1 (error).
+    auto find_stop = [&](int t) -> int {
+      for (int sb = t - 2 < 0 ? 0 : t - 2; sb < t; ++sb) {
+        if (!warp_all(tc::mbar_wait(&c.decided[sb & 1], (sb >> 1) & 1, abort_flag, dev_status))) return -1;
+        if (c.stop_at == sb) return sb;
+      }
+      return -1;
+    };
+    // the result is O^(sb) for a stop on block sb: the saved copy when sb = t-2, else the
+    // current O (folded through t-1)
+    auto take = [&](int sb, int t) {
+      if (sb == t - 2) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) { o[h] = o_sv[h]; lw[h] = l_sv[h]; }
+      }
+      used = sb + 1;
+    };
     if (ns > 0) ok = softmax(0, a_cur, p_cur) == 0;  // an empty visit list leaves O = 0
     for (int t = 0; ok && t < ns; ++t) {
       const int buf = t & 1;
       if (t + 1 < ns) {
-        const int r = softmax(t + 1, a_nxt, p_nxt);   // P_{t+1} while PV_t runs
-        if (r == 1) {
-          // halted before S_{t+1}: only a stop decided on block t-1 does that; then
-          // O^(t-1) (already folded) is the result and PV_t is not needed
-          ok = t >= 1 && warp_all(tc::mbar_wait(&c.decided, (t - 1) & 1, abort_flag, dev_status)) &&
-               c.stop_at == t - 1;
-          if (ok) used = t;
+        const int rs = softmax(t + 1, a_nxt, p_nxt);  // P_{t+1} while PV_t runs
+        if (rs == 1) {
+          // halted before S_{t+1}: a stop was decided on block t-2 or t-1
+          const int sb = find_stop(t);
+          ok = sb >= 0;
+          if (ok) take(sb, t);
           break;
         }
-        ok = r == 0;
+        ok = rs == 0;
         if (!ok) break;
       }
+      // PV_t is issued: P_t was published, and the MMA issuer only skips it once this loop
+      // has ended
       ok = warp_all(tc::mbar_wait(&c.o_full[buf], (t >> 1) & 1, abort_flag, dev_status));
       if (!ok) break;
       tc::tc_fence_after();
       uint32_t dv[16];
       tc::tmem_ld16(tl + 32 + buf * NPAD, dv);
       tc::tc_fence_before();
-      if (t >= 1) {
-        // the verdict on block t-1 (usually long made): on a stop, O^(t-1) is final
-        ok = warp_all(tc::mbar_wait(&c.decided, (t - 1) & 1, abort_flag, dev_status));
+      if (t >= 2) {
+        // the verdict on block t-2 (it also frees that block's probe slot, reused below)
+        ok = warp_all(tc::mbar_wait(&c.decided[buf], ((t - 2) >> 1) & 1, abort_flag, dev_status));
         if (!ok) break;
-        if (c.stop_at == t - 1) {
-          used = t;
+        if (c.stop_at == t - 2) {
+          take(t - 2, t);
           break;
         }
       }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
+        o_sv[h] = o[h];
+        l_sv[h] = lw[h];
         o[h] = fmaf(o[h], a_cur[h], __uint_as_float(dv[h]));
         lw[h] = fmaf(lw[h], a_cur[h], p_cur[h]);
         a_cur[h] = a_nxt[h];
@@ -336,7 +372,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       c.xfull[buf][r] = o[0];
       if (lane == 0) c.lpart[buf][quarter] = lw[0];
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&c.probe_rdy);
+      if (lane == 0) tc::mbar_arrive(&c.probe_rdy[buf]);
+    }
+    if (ok && used == ns && ns >= 2) {
+      // every block was folded; the verdict on block ns-2 is still unread (one on ns-1
+      // would leave the result as it is)
+      const int sb = ns - 2;
+      ok = warp_all(tc::mbar_wait(&c.decided[sb & 1], (sb >> 1) & 1, abort_flag, dev_status));
+      if (ok && c.stop_at == sb) take(sb, ns);
     }
 #pragma unroll
     for (int h = 1; h < G; ++h) {
@@ -348,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
       for (int h = 0; h < G; ++h) c.lfin[quarter][h] = lw[h];
     }
     if (threadIdx.x == 64) {
+      *sm_quit = 1;
       *halt = 1;                       // nothing more to stream
       blocks_used[bg] = ok ? used : 0;
     }
@@ -358,18 +402,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
   } else if (warp == 6) {
     // ---------------- decider ----------------
     // Lane i owns probe coordinates i and i + 32: it forms x = O / l for them (the
-    // fp32 divisions run in parallel), writes the trace, and the exact fp64 products
-    // x_t^2 and x_t x_{t-1} (products of fp32 values are exact in fp64). Lane 0 adds
-    // them up in coordinate order, then tests stability; ||x_{t-1}||^2 and its root are
-    // the previous block's, the same sum in the same order.
+    // fp32 divisions run in parallel), writes the trace, and the fp64 products x_t^2 and
+    // x_t x_{t-1} (exact: products of fp32 values). The sums run across the warp in the
+    // fixed pairwise order of warp_pairwise_sum; every lane then holds them and takes the
+    // same decision. ||x_{t-1}|| is the previous block's root (the same sum of the same
+    // values).
     const int np = a.n_probe;
     const int d0 = lane < np ? a.dims[lane] : 0;
     const int d1 = lane + 32 < np ? a.dims[lane + 32] : 0;
     float xp0 = 0.f, xp1 = 0.f;
-    double np_prev = 0.0;          // lane 0: ||x_{t-1}||
+    double np_prev = 0.0;          // ||x_{t-1}||
     int run = 0;
     for (int t = 0; t < ns; ++t) {
-      if (!warp_all(tc::mbar_wait(&c.probe_rdy, t & 1, abort_flag, dev_status))) break;
+      if (!warp_all(tc::mbar_wait(&c.probe_rdy[t & 1], (t >> 1) & 1, abort_flag, dev_status))) break;
       const int buf = t & 1;
       const float lt = (c.lpart[buf][0] + c.lpart[buf][1]) + (c.lpart[buf][2] + c.lpart[buf][3]);
       const float x0 = lane < np ? __fdiv_rn(c.xfull[buf][d0], lt) : 0.f;
@@ -379,42 +424,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(
         if (lane < np) tr[lane] = x0;
         if (lane + 32 < np) tr[lane + 32] = x1;
       }
-      c.prod[0][lane] = __dmul_rn((double)x0, (double)x0);
-      c.prod[1][lane] = __dmul_rn((double)x0, (double)xp0);
-      c.prod[0][lane + 32] = __dmul_rn((double)x1, (double)x1);
-      c.prod[1][lane + 32] = __dmul_rn((double)x1, (double)xp1);
+      const double sc2 = warp_pairwise_sum(
+          __dadd_rn(__dmul_rn((double)x0, (double)x0), __dmul_rn((double)x1, (double)x1)));
+      const double dt = warp_pairwise_sum(
+          __dadd_rn(__dmul_rn((double)x0, (double)xp0), __dmul_rn((double)x1, (double)xp1)));
       xp0 = x0;
       xp1 = x1;
-      __syncwarp();
+      const double nc = __dsqrt_rn(sc2);
+      bool stop = false;
+      if (t >= 1) {
+        const double ds = fabs(__dadd_rn(nc, -np_prev));
+        const double den = __dmul_rn(nc, np_prev);
+        const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
+        const bool stable = (ds < (double)a.tau) && (dd < (double)a.phi);
+        run = stable ? run + 1 : 0;
+        stop = a.enable && run >= a.patience;
+      }
+      np_prev = nc;
       if (lane == 0) {
-        bool stop = false;
-        double sc2 = 0.0, dt = 0.0;
-        if (t >= 1) {
-          for (int i = 0; i < np; ++i) {
-            sc2 = __dadd_rn(sc2, c.prod[0][i]);
-            dt = __dadd_rn(dt, c.prod[1][i]);
-          }
-        } else {
-          for (int i = 0; i < np; ++i) sc2 = __dadd_rn(sc2, c.prod[0][i]);
-        }
-        const double nc = __dsqrt_rn(sc2), npv = np_prev;
-        np_prev = nc;
-        if (t >= 1) {
-          const double ds = fabs(__dadd_rn(nc, -npv));
-          const double den = __dmul_rn(nc, npv);
-          const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
-          const bool stable = (ds < (double)a.tau) && (dd < (double)a.phi);
-          run = stable ? run + 1 : 0;
-          stop = a.enable && run >= a.patience;
-        }
         if (stop) {
           c.stop_at = t;
           *halt = 1;                    // release the producer and the MMA issuer
         }
-        tc::mbar_arrive(&c.decided);
+        tc::mbar_arrive(&c.decided[t & 1]);
       }
-      __syncwarp();
-      if (c.stop_at == t) break;
+      if (stop) break;
     }
   }
 

@@ -133,7 +133,9 @@ typedef struct {
 /* Run-time termination ([ART] 2.2-2.4).
  *   tau, phi     thresholds: block t >= 1 is stable iff |‖x_t‖-‖x_{t-1}‖| < tau and
  *                1 - cos(x_t, x_{t-1}) < phi (1 when a norm is 0), computed in fp64
- *                on the fp32 probe values with sums in index order.
+ *                on the fp32 probe values: exact products, each sum over the
+ *                coordinates in one fixed pairwise order (coordinate i with i + 32,
+ *                zero where absent, then values 16, 8, 4, 2, 1 apart).
  *   patience     stop after `patience` consecutive stable blocks (>= 1) ([ART] 2.3).
  *   enable       0 = never stop (probes are still recorded when asked for).
  *   n_probe      number of probe coordinates (1..64).

@@ -464,20 +464,34 @@ def attend_vs(Q, K, V, v_idx, v_cnt, s_off, s_cnt, scale, rows=None):
 # ---------------------------------------------------------------------------
 # a8: decode with run-time termination
 
+def pairwise_sum64(terms) -> float:
+    """Sum of at most 64 fp64 terms in one fixed pairwise order, each add rounded
+    (IEEE, to nearest): term i is added to term i + 32 (zero where there is none),
+    then values 16, 8, 4, 2 and 1 apart. The pages give no order for the probe
+    sums of [ART, 2.2]; this one is the reading chosen (a warp of 32 lanes holding
+    two coordinates each evaluates it in five steps)."""
+    t = np.asarray(terms, dtype=np.float64)
+    assert t.ndim == 1 and t.size <= 64
+    a = np.zeros(64)
+    a[:t.size] = t
+    a = a[:32] + a[32:]
+    while a.size > 1:
+        h = a.size // 2
+        a = a[:h] + a[h:]
+    return float(a[0])
+
+
 def probe_step(x_prev: Sequence[float], x_cur: Sequence[float]):
     """(d_scale, d_direction) between consecutive probes ([ART, 2.2]):
     the absolute difference of their L2 norms and one minus their cosine.
-    fp64 on the fp32 probe values; every sum runs in index order with a
-    separate multiply and add; d_direction = 1 when a norm is zero."""
-    s_cur = 0.0
-    s_prev = 0.0
-    dot = 0.0
-    for a, b in zip(x_cur, x_prev):
-        a = float(a)
-        b = float(b)
-        s_cur = s_cur + a * a
-        s_prev = s_prev + b * b
-        dot = dot + a * b
+    fp64 on the fp32 probe values (at most 64): products rounded on their own
+    (exact, being products of fp32 values), sums in the pairwise order of
+    pairwise_sum64; d_direction = 1 when a norm is zero."""
+    xc = np.asarray(x_cur, dtype=np.float32).astype(np.float64)
+    xp = np.asarray(x_prev, dtype=np.float32).astype(np.float64)
+    s_cur = pairwise_sum64(xc * xc)
+    s_prev = pairwise_sum64(xp * xp)
+    dot = pairwise_sum64(xc * xp)
     n_cur = math.sqrt(s_cur)
     n_prev = math.sqrt(s_prev)
     d_scale = abs(n_cur - n_prev)

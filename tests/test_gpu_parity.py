@@ -199,6 +199,18 @@ def test_decode_limits():
     assert (used == 32).all()
 
 
+@pytest.mark.parametrize("nb", [1, 2, 3, 4, 7])
+def test_decode_stop_on_each_late_block(nb):
+    """A stop on every block of short caches, the last two included: the kernel reads the
+    verdict on a block two blocks later, so a stop on the next-to-last block is settled
+    after its loop, one on the last block leaves the full result, and a stop seen as a
+    halt before the next score block arrives is traced back to its block."""
+    spec = S.DECODE_WORKLOADS["decode_art_64k"].scaled(B=2, L=128 * nb)
+    for p in range(1, nb + 1):
+        used, _ = _check_decode(spec, 1014, float("inf"), float("inf"), p)
+        assert (used == min(p + 1, nb)).all(), (nb, p, used)
+
+
 @pytest.mark.parametrize("Hq,Hkv,d,bkv", [(8, 1, 128, 128), (4, 4, 64, 64), (8, 4, 128, 64)])
 def test_decode_shapes(Hq, Hkv, d, bkv):
     spec = S.DecodeSpec("dec", B=2, Hq=Hq, Hkv=Hkv, L=2048, d=d, block_kv=bkv, tau=1e-2,

@@ -409,6 +409,55 @@ def test_probe_step_values():
     assert ds == 0.0 and dd == 2.0
 
 
+def test_pairwise_sum64_order_and_bound():
+    """The probe sums follow the stated pairwise order. Worked by hand: with terms
+    1 (index 0), 2^-53 (index 1) and 2^-53 (index 33), index 1 and index 33 meet
+    first (2^-52, exact) and the last step gives 1 + 2^-52, while a left-to-right sum
+    rounds each 2^-53 away (ties to even) and returns 1."""
+    t = np.zeros(34)
+    t[0], t[1], t[33] = 1.0, 2.0 ** -53, 2.0 ** -53
+    assert O.pairwise_sum64(t) == 1.0 + 2.0 ** -52
+    left = 0.0
+    for v in t:
+        left += v
+    assert left == 1.0
+    # index 0 with index 32 first: 1 + 2^-53 rounds to 1 there
+    t = np.zeros(64)
+    t[0], t[32], t[1] = 1.0, 2.0 ** -53, 2.0 ** -53
+    assert O.pairwise_sum64(t) == 1.0
+    # exact rational sums: a tree of depth 6 is within 6 u sum|t| of the exact value,
+    # and exact when every partial sum is representable (small integers)
+    from fractions import Fraction
+    rng = np.random.default_rng(3)
+    for n in (1, 2, 31, 32, 33, 64):
+        x = rng.standard_normal(n).astype(np.float32).astype(np.float64)
+        terms = x * x
+        exact = sum(Fraction(float(v)) for v in terms)
+        got = O.pairwise_sum64(terms)
+        bound = 6 * 2.0 ** -53 * float(sum(abs(Fraction(float(v))) for v in terms)) * 1.0001
+        assert abs(Fraction(got) - exact) <= Fraction(bound), n
+        ints = rng.integers(-1000, 1000, size=n).astype(np.float64)
+        assert O.pairwise_sum64(ints) == float(ints.sum())
+
+
+def test_probe_step_matches_exact_arithmetic():
+    """d_scale and d_direction from random fp32 probes against the same quantities
+    in exact rational arithmetic (the roots and the quotient within a few units of
+    fp64 rounding)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(4)
+    for n in (1, 7, 32, 64):
+        a = rng.standard_normal(n).astype(np.float32)
+        b = (a + 0.01 * rng.standard_normal(n)).astype(np.float32)
+        ds, dd = O.probe_step(a, b)
+        sa = sum(Fraction(float(v)) ** 2 for v in a)
+        sb = sum(Fraction(float(v)) ** 2 for v in b)
+        dot = sum(Fraction(float(u)) * Fraction(float(v)) for u, v in zip(a, b))
+        na, nb = math.sqrt(float(sa)), math.sqrt(float(sb))
+        assert abs(ds - abs(nb - na)) <= 1e-14 * max(na, nb)
+        assert abs(dd - (1 - float(dot) / (na * nb))) <= 1e-14
+
+
 def _decode_case(seed=11, L=2048, d=128, G=4, bkv=128):
     rng = np.random.default_rng(seed)
     q = S.f32_to_bf16_bits(rng.standard_normal((G, d)).astype(np.float32))
