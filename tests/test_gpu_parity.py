@@ -199,7 +199,7 @@ def test_decode_limits():
     assert (used == 32).all()
 
 
-@pytest.mark.parametrize("nb", [1, 2, 3, 4, 7])
+@pytest.mark.parametrize("nb", [1, 2, 3, 4, 5, 7, 9])
 def test_decode_stop_on_each_late_block(nb):
     """A stop on every block of short caches, the last two included: the kernel reads the
     verdict on a block two blocks later, so a stop on the next-to-last block is settled
