@@ -189,10 +189,10 @@ bsa_status run_score(const bsa_shape& s, bsa_score_kind kind, float beta, const 
                      const void* v, float* scores, int32_t* dev_status, const ScoreWs& w, cudaStream_t cs) {
   cudaError_t e;
   if (kind == BSA_SCORE_KMINMAX) {
-    const bool tc = bsa::score_tc_supported(s);
+    const bool tc = bsa::score_rank_supported(s);
     e = bsa::launch_pool_bounds(s, k, w.kbar, w.kbar2, tc ? w.h16 : nullptr, w.h16b, w.kinv, cs);
     if (e != cudaSuccess) return cuda_fail(e, "pool (bounds)");
-    e = tc ? bsa::launch_score_tc_bounds(s, q, w.h16, w.h16b, w.kinv, scores, dev_status, cs)
+    e = tc ? bsa::launch_score_rank_bounds(s, q, w.h16, w.h16b, w.kinv, scores, dev_status, cs)
            : bsa::launch_score_simt(s, q, w.kbar, w.kbar2, nullptr, 0, scores, cs);
     if (e != cudaSuccess) return cuda_fail(e, tc ? "score (tensor cores)" : "score");
     return BSA_OK;
@@ -543,7 +543,7 @@ int bsa_attend_path(const bsa_shape* s, int W) {
 
 int bsa_score_path(const bsa_shape* s, bsa_score_kind kind) {
   if (check_shape(s) != BSA_OK || !known_kind(kind)) return -1;
-  const bool tc = kind == BSA_SCORE_KMINMAX ? bsa::score_tc_supported(*s) : bsa::score_rank_supported(*s);
+  const bool tc = bsa::score_rank_supported(*s);
   return tc ? BSA_PATH_TENSOR_CORES : BSA_PATH_CUDA_CORES;
 }
 

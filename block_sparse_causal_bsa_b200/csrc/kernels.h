@@ -28,13 +28,6 @@ cudaError_t launch_score_simt(const bsa_shape& s, const void* q, const float* kb
                               const float* kbar2, const float* wnorm, int wmode, float* scores,
                               cudaStream_t st);
 
-// K-min/K-max block scores on tcgen05 tensor cores (bf16 inputs; mid16/rad16/kinv from
-// launch_pool_bounds).
-bool score_tc_supported(const bsa_shape& s);
-cudaError_t launch_score_tc_bounds(const bsa_shape& s, const void* q, const uint16_t* mid16,
-                                   const uint16_t* rad16, const float* kinv, float* scores,
-                                   int32_t* dev_status, cudaStream_t st);
-
 // Mean-pooled block scores on tcgen05 (fp16 operands with power-of-two scales), persistent,
 // optionally fused with the ranking of the selection. kbar16/kinv from launch_pool.
 // ranked == null: scores only (scores required). ranked != null: also the top-M lists
@@ -42,6 +35,11 @@ cudaError_t launch_score_tc_bounds(const bsa_shape& s, const void* q, const uint
 // ring [ring_ctas][kScoreRankRing][heads per unit][n_kb] instead (the grid is capped at
 // ring_ctas).
 bool score_rank_supported(const bsa_shape& s);
+// The K-min/K-max backbone in the same persistent kernel (one head per unit, two passes per
+// chunk: mid against Q, rad against |Q|); mid16, rad16, kinv from launch_pool_bounds.
+cudaError_t launch_score_rank_bounds(const bsa_shape& s, const void* q, const uint16_t* mid16,
+                                     const uint16_t* rad16, const float* kinv, float* scores,
+                                     int32_t* dev_status, cudaStream_t st);
 bool score_rank_fusable(const bsa_shape& s);          // the ranking too
 int score_rank_heads_per_unit(const bsa_shape& s);
 constexpr int kScoreRankRingCtas = 256;

@@ -17,6 +17,13 @@
 // unless an element lies more than 2^-24 below the tile's largest) and the fp32
 // accumulation; the epilogue multiplies the row max by 2^-s and 2^-r, again exactly.
 //
+// The K-min/K-max backbone ([UGS] Metodologia step 1, per-coordinate upper bounds) runs
+// in the same kernel (BOUNDS): s(t,j) = max over rows of sum_c max(q_c kmin_jc, q_c kmax_jc)
+// = q . mid_j + |q| . rad_j with mid = (kmin+kmax)/2 and rad = (kmax-kmin)/2 >= 0, so each
+// chunk is two fp16 passes into one accumulator, mid against Q and rad against |Q| (written
+// by the conversion beside Q). One head per unit: two heads' Q and |Q|, double-buffered,
+// would not fit in shared memory.
+//
 // Persistent: one CTA per SM walks units (batch, KV head, query tile, head pair),
 // longest tiles first. Warps:
 //   0 (one thread)  TMA: each unit's query tiles (bf16) into one of two Q buffers,
@@ -57,12 +64,13 @@ constexpr uint32_t kChunk = 2 * kHalfTile;    // one pooled-key chunk (128 block
 constexpr int kRankWarpsF = 5;                // rank warps of the fused kernel
 constexpr int kRing = kScoreRankRing;         // units whose rows the L2 ring holds
 
-template <int HP, bool RANK>
+template <int HP, bool RANK, bool BOUNDS>
 struct SRLayout {
   static constexpr int rank_warps = RANK ? kRankWarpsF : 0;
   static constexpr int threads = (2 + kEpiWarps + rank_warps) * 32;
   static constexpr uint32_t qhalf = HP * kHalfTile;     // one d-half of all HP heads' tiles
-  static constexpr uint32_t qbuf = 2 * qhalf;           // one Q buffer
+  static constexpr uint32_t qabs = 2 * qhalf;           // K-min/K-max: |Q| behind Q in the buffer
+  static constexpr uint32_t qbuf = (BOUNDS ? 2 : 1) * 2 * qhalf;   // one Q buffer
   static constexpr size_t smem_q = 0;                   // two Q buffers
   static constexpr size_t smem_k = 2 * (size_t)qbuf;    // two chunk stages
   static constexpr size_t smem_rank = smem_k + 2 * (size_t)kChunk;
@@ -129,10 +137,17 @@ __device__ __forceinline__ void unit_coords(int u, int npair, int BG, int n_qt, 
 }
 }  // namespace
 
-template <int HP, bool RANK>
-__global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_kernel(
-    const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk, const SRArgs a) {
-  using L = SRLayout<HP, RANK>;
+// BOUNDS: the K-min/K-max backbone (one head per unit, no ranking). tmk then holds the
+// per-block mid = (kmin+kmax)/2 and tmk2 the rad = (kmax-kmin)/2 >= 0 (fp16, one power-of-two
+// scale per block, as for the mean), and each chunk is two passes into one accumulator,
+// mid against Q and rad against |Q|: sum_c max(q_c kmin_c, q_c kmax_c) = q . mid + |q| . rad.
+template <int HP, bool RANK, bool BOUNDS>
+__global__ void __launch_bounds__(SRLayout<HP, RANK, BOUNDS>::threads, 1) score_rank_kernel(
+    const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+    const __grid_constant__ CUtensorMap tmk2, const SRArgs a) {
+  static_assert(!BOUNDS || (HP == 1 && !RANK), "the K-min/K-max variant scores one head per unit");
+  using L = SRLayout<HP, RANK, BOUNDS>;
+  constexpr int kParts = BOUNDS ? 2 : 1;        // pooled-key half-chunks per chunk
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   SRCtrl<HP>& c = *reinterpret_cast<SRCtrl<HP>*>(sm + L::smem_ctrl);
@@ -180,6 +195,7 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
     // ---------------- TMA producer ----------------
     tc::prefetch_tmap(&tmq);
     tc::prefetch_tmap(&tmk);
+    if (BOUNDS) tc::prefetch_tmap(&tmk2);
     auto issue_q = [&](int li, int u) -> bool {
       const int qb = li & 1;
       if (li >= 2 && !tc::mbar_wait(&c.q_empty[qb], ((li >> 1) - 1) & 1, abort_flag, dev_status)) return false;
@@ -188,7 +204,7 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
       const int b = bg / a.Hkv, g = bg % a.Hkv;
       const int h0 = g * G + pr * HP;
       uint8_t* dst = sm + L::smem_q + qb * L::qbuf;
-      tc::mbar_arrive_expect_tx(&c.q_full[qb], L::qbuf);
+      tc::mbar_arrive_expect_tx(&c.q_full[qb], 2 * L::qhalf);   // the bf16 tiles (|Q| is made here)
       for (int hp = 0; hp < HP; ++hp) {
         const int qrow = (int)(((size_t)b * a.Hq + h0 + hp) * a.N + (size_t)t * TQ);
         tc::tma_load_2d(dst + hp * kHalfTile, &tmq, 0, qrow, &c.q_full[qb]);
@@ -198,36 +214,36 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
       return true;
     };
     bool ok = (int)blockIdx.x >= a.units || issue_q(0, blockIdx.x);
-    int gc = 0;
+    int gk = 0;                                   // half-chunk loads (one per chunk unless BOUNDS)
     for (int li = 0, u = blockIdx.x; ok && u < a.units; ++li, u += stride) {
       int t, bg, pr;
       unit_coords(u, npair, BG, a.n_qt, t, bg, pr);
       const int J = (int)(((long long)(t + 1) * TQ - 1) / a.block_k);
       const int nc = (J + 1 + CB - 1) / CB;
-      for (int ch = 0; ch < nc; ++ch, ++gc) {
-        const int s = gc & 1;
-        if (gc >= 2 && !tc::mbar_wait(&c.kb_empty[s], ((gc >> 1) - 1) & 1, abort_flag, dev_status)) {
-          ok = false;
-          break;
+      for (int ch = 0; ok && ch < nc; ++ch) {
+        for (int part = 0; part < kParts; ++part, ++gk) {
+          const int s = gk & 1;
+          if (gk >= 2 && !tc::mbar_wait(&c.kb_empty[s], ((gk >> 1) - 1) & 1, abort_flag, dev_status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = sm + L::smem_k + s * kChunk;
+          const int row = bg * a.n_kb + ch * CB;
+          const CUtensorMap* m = part ? &tmk2 : &tmk;
+          tc::mbar_arrive_expect_tx(&c.kb_full[s], kChunk);
+          tc::tma_load_2d(dst, m, 0, row, &c.kb_full[s]);
+          tc::tma_load_2d(dst + kHalfTile, m, 64, row, &c.kb_full[s]);
+          kb_issued = gk + 1;
         }
-        uint8_t* dst = sm + L::smem_k + s * kChunk;
-        const int row = bg * a.n_kb + ch * CB;
-        tc::mbar_arrive_expect_tx(&c.kb_full[s], kChunk);
-        tc::tma_load_2d(dst, &tmk, 0, row, &c.kb_full[s]);
-        tc::tma_load_2d(dst + kHalfTile, &tmk, 64, row, &c.kb_full[s]);
-        kb_issued = gc + 1;
         // the next unit's query tiles, as soon as their buffer is free
-        if (ch == 0 && u + stride < a.units && !issue_q(li + 1, u + stride)) {
-          ok = false;
-          break;
-        }
+        if (ok && ch == 0 && u + stride < a.units && !issue_q(li + 1, u + stride)) ok = false;
       }
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
     constexpr uint32_t idesc = tc::idesc_f16_f32(CB, HP * TQ, false, false);
     bool ok = true;
-    int gc = 0;
+    int gc = 0, gk = 0;
     for (int li = 0, u = blockIdx.x; ok && u < a.units; ++li, u += stride) {
       const int qb = li & 1;
       if (!tc::mbar_wait(&c.qc_full[qb], (li >> 1) & 1, abort_flag, dev_status)) break;
@@ -237,22 +253,27 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
       const int nc = (J + 1 + CB - 1) / CB;
       const uint32_t qbase = sQ + qb * L::qbuf;
       for (int ch = 0; ch < nc; ++ch, ++gc) {
-        const int db = gc & 1, s = gc & 1;
-        ok = (gc < 2 || tc::mbar_wait(&c.d_free[db], ((gc >> 1) - 1) & 1, abort_flag, dev_status)) &&
-             tc::mbar_wait(&c.kb_full[s], (gc >> 1) & 1, abort_flag, dev_status);
-        if (!ok) break;
-        tc::tc_fence_after();
-        const uint32_t kb = sK + s * kChunk;
+        const int db = gc & 1;
+        ok = gc < 2 || tc::mbar_wait(&c.d_free[db], ((gc >> 1) - 1) & 1, abort_flag, dev_status);
         const uint32_t d = tmem + db * L::dcols;
+        for (int part = 0; ok && part < kParts; ++part, ++gk) {
+          const int s = gk & 1;
+          ok = tc::mbar_wait(&c.kb_full[s], (gk >> 1) & 1, abort_flag, dev_status);
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint32_t kb = sK + s * kChunk;
+          const uint32_t qpart = qbase + (part ? L::qabs : 0u);   // Q against mid, |Q| against rad
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * kHalfTile + (kk & 3) * 32;
-          const uint32_t boff = (kk >> 2) * L::qhalf + (kk & 3) * 32;
-          tc::umma_bf16(d, tc::sdesc_sw128(kb + aoff, 16, 1024), tc::sdesc_sw128(qbase + boff, 16, 1024),
-                        idesc, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (kk >> 2) * kHalfTile + (kk & 3) * 32;
+            const uint32_t boff = (kk >> 2) * L::qhalf + (kk & 3) * 32;
+            tc::umma_bf16(d, tc::sdesc_sw128(kb + aoff, 16, 1024), tc::sdesc_sw128(qpart + boff, 16, 1024),
+                          idesc, (part > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_issued = true;
+          tc::umma_commit(&c.kb_empty[s]);
         }
-        mma_issued = true;
-        tc::umma_commit(&c.kb_empty[s]);
+        if (!ok) break;
         tc::umma_commit(&c.d_full[db]);
       }
       if (!ok) break;
@@ -317,8 +338,11 @@ __global__ void __launch_bounds__(SRLayout<HP, RANK>::threads, 1) score_rank_ker
             w4[e] = *reinterpret_cast<const uint32_t*>(&h2);
           }
           const int half = p >> 3, ck = (p & 7) ^ (r & 7);
-          *reinterpret_cast<uint4*>(base + half * L::qhalf + hp * kHalfTile + r * 128 + ck * 16) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          const uint32_t off = half * L::qhalf + hp * kHalfTile + r * 128 + ck * 16;
+          *reinterpret_cast<uint4*>(base + off) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          if (BOUNDS)        // |Q| in fp16: the same values with the sign bits cleared
+            *reinterpret_cast<uint4*>(base + L::qabs + off) =
+                make_uint4(w4[0] & 0x7fff7fffu, w4[1] & 0x7fff7fffu, w4[2] & 0x7fff7fffu, w4[3] & 0x7fff7fffu);
         }
       }
       tc::fence_proxy_async_smem();               // generic writes -> tensor-core reads
@@ -504,16 +528,24 @@ bool score_rank_fusable(const bsa_shape& s) { return score_rank_supported(s); }
 
 int score_rank_heads_per_unit(const bsa_shape& s) { return ((s.Hq / s.Hkv) % 2 == 0) ? 2 : 1; }
 
-template <int HP, bool RANK>
+template <int HP, bool RANK, bool BOUNDS = false>
 static cudaError_t launch_sr(const bsa_shape& s, const CUtensorMap& mq, const CUtensorMap& mk,
-                             const SRArgs& a, int grid, cudaStream_t st) {
-  using L = SRLayout<HP, RANK>;
+                             const CUtensorMap& mk2, const SRArgs& a, int grid, cudaStream_t st) {
+  using L = SRLayout<HP, RANK, BOUNDS>;
   const size_t smem = L::smem_ctrl + sizeof(SRCtrl<HP>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(score_rank_kernel<HP, RANK>,
+  static_assert(L::smem_ctrl + sizeof(SRCtrl<HP>) + 1024 <= 227 * 1024, "shared memory");
+  cudaError_t e = cudaFuncSetAttribute(score_rank_kernel<HP, RANK, BOUNDS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  score_rank_kernel<HP, RANK><<<grid, L::threads, smem, st>>>(mq, mk, a);
+  score_rank_kernel<HP, RANK, BOUNDS><<<grid, L::threads, smem, st>>>(mq, mk, mk2, a);
   return cudaGetLastError();
+}
+
+static int sm_count(int* sms) {
+  int dev = 0;
+  *sms = 148;
+  return cudaGetDevice(&dev) == cudaSuccess &&
+         cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess;
 }
 
 cudaError_t launch_score_rank(const bsa_shape& s, const bsa_select_params* p, const void* q,
@@ -548,16 +580,48 @@ cudaError_t launch_score_rank(const bsa_shape& s, const bsa_select_params* p, co
   a.block_k = s.block_k;
   const long long units = (long long)s.B * s.Hkv * n_qt * ((s.Hq / s.Hkv) / HP);
   a.units = (int)units;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return cudaErrorInvalidValue;
+  int sms = 148;
+  if (!sm_count(&sms)) return cudaErrorInvalidValue;
   long long grid = units < sms ? units : sms;
   if (ranked && !scores && grid > ring_ctas) grid = ring_ctas;
   if (grid < 1) grid = 1;
   if (ranked) {
-    return HP == 2 ? launch_sr<2, true>(s, mq, mk, a, (int)grid, st) : launch_sr<1, true>(s, mq, mk, a, (int)grid, st);
+    return HP == 2 ? launch_sr<2, true>(s, mq, mk, mk, a, (int)grid, st)
+                   : launch_sr<1, true>(s, mq, mk, mk, a, (int)grid, st);
   }
-  return HP == 2 ? launch_sr<2, false>(s, mq, mk, a, (int)grid, st) : launch_sr<1, false>(s, mq, mk, a, (int)grid, st);
+  return HP == 2 ? launch_sr<2, false>(s, mq, mk, mk, a, (int)grid, st)
+                 : launch_sr<1, false>(s, mq, mk, mk, a, (int)grid, st);
+}
+
+cudaError_t launch_score_rank_bounds(const bsa_shape& s, const void* q, const uint16_t* mid16,
+                                     const uint16_t* rad16, const float* kinv, float* scores,
+                                     int32_t* dev_status, cudaStream_t st) {
+  CUtensorMap mq, mm, mr;
+  const uint64_t qrows = (uint64_t)s.B * s.Hq * s.N;
+  const uint64_t krows = (uint64_t)s.B * s.Hkv * (s.N / s.block_k);
+  if (!make_tmap_bf16_2d(&mq, q, qrows, HD, 64, TQ) || !make_tmap_bf16_2d(&mm, mid16, krows, HD, 64, CB) ||
+      !make_tmap_bf16_2d(&mr, rad16, krows, HD, 64, CB))
+    return cudaErrorInvalidValue;
+  const int n_qt = s.N / TQ;
+  SRArgs a{};
+  a.kinv = kinv;
+  a.wmode = 0;
+  a.scores = scores;
+  a.rho = 1;
+  a.dev_status = dev_status;
+  a.N = s.N;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.n_qt = n_qt;
+  a.n_kb = s.N / s.block_k;
+  a.block_k = s.block_k;
+  const long long units = (long long)s.B * s.Hkv * n_qt * (s.Hq / s.Hkv);
+  a.units = (int)units;
+  int sms = 148;
+  if (!sm_count(&sms)) return cudaErrorInvalidValue;
+  long long grid = units < sms ? units : sms;
+  if (grid < 1) grid = 1;
+  return launch_sr<1, false, true>(s, mq, mm, mr, a, (int)grid, st);
 }
 
 }  // namespace bsa

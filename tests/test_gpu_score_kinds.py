@@ -18,7 +18,7 @@ from block_sparse_causal_bsa_b200 import binding as bb
 from block_sparse_causal_bsa_b200 import synthetic as S
 from oracle import bsa_oracle as O
 
-from gpu_util import check_attend, check_scores, check_selection, inputs, out_rows
+from gpu_util import check_attend, check_scores, check_selection, inputs, out_rows, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -59,6 +59,45 @@ def test_kminmax_tensor_core():
     spec = S.WORKLOADS["gated_prefill_128k"].scaled(N=4096, Hq=8, Hkv=2, k_first=12, k_last=12)
     g, ref_sel = _run(spec, 1502, "kminmax")
     assert ref_sel["trigger"].sum() > 0
+
+
+@pytest.mark.parametrize("N,Hq,Hkv,bk", [(16384, 4, 1, 64), (32768, 2, 2, 128)])
+def test_kminmax_scores_several_chunks(N, Hq, Hkv, bk):
+    """K-min/K-max scores of whole layers whose late tiles span two chunks of 128 blocks,
+    with several units per persistent CTA, one and four query heads per KV head."""
+    spec = S.PrefillSpec("kmm", B=1, Hq=Hq, Hkv=Hkv, N=N, d=128, block_k=bk, tile_q=128,
+                         k_first=8, k_last=8, rho=2, gate_quantile=0.25, score_kind="mean",
+                         dtype="bf16", structure="twins", p_twin=0.36)
+    (q, k, _), (qd, kd, _) = inputs(spec, 1504)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g = bb.score(qd, kd, block_k=bk, tile_q=128, kind="kminmax", status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    check_scores(g.cpu().numpy(), O.block_scores(q, k, 128, bk, kind="bounds"))
+
+
+def test_kminmax_scores_full_size_sampled():
+    """The 128k gated workload's K-min/K-max scores on sampled rows (the first and last
+    tiles included) against the oracle's per-row bound."""
+    spec = S.WORKLOADS["gated_prefill_128k"]
+    q, k, _ = S.prefill_inputs(spec, 1505)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g = bb.score(to_dev(q), to_dev(k), block_k=spec.block_k, tile_q=spec.tile_q, kind="kminmax",
+                 status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    G = spec.Hq // spec.Hkv
+    rng = np.random.default_rng(1505)
+    rows = [(0, 0, 0), (spec.B - 1, spec.Hq - 1, spec.n_qt - 1)] + [
+        (int(rng.integers(spec.B)), int(rng.integers(spec.Hq)), int(rng.integers(spec.n_qt))) for _ in range(6)]
+    bounds = {}
+    for b, h, t in rows:
+        if (b, h // G) not in bounds:
+            bounds[b, h // G] = O.key_block_bounds(k[b, h // G], spec.block_k)
+        kmin, kmax = bounds[b, h // G]
+        _, J = O.tile_blocks(t, spec.tile_q, spec.block_k)
+        ref = O.score_tile_bounds(q[b, h, t * spec.tile_q:(t + 1) * spec.tile_q], kmin, kmax, J)
+        check_scores(g[b, h, t].cpu().numpy()[None], ref[None])
 
 
 @pytest.mark.parametrize("kind", ["vlog", "kminmax"])
