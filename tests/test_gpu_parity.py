@@ -211,8 +211,10 @@ def test_decode_stop_on_each_late_block(nb):
         assert (used == min(p + 1, nb)).all(), (nb, p, used)
 
 
-@pytest.mark.parametrize("Hq,Hkv,d,bkv", [(8, 1, 128, 128), (4, 4, 64, 64), (8, 4, 128, 64)])
+@pytest.mark.parametrize("Hq,Hkv,d,bkv", [(8, 1, 128, 128), (2, 2, 128, 128), (4, 2, 128, 128),
+                                          (4, 4, 64, 64), (8, 4, 128, 64)])
 def test_decode_shapes(Hq, Hkv, d, bkv):
+    """Group sizes 8, 1 and 2 on the tensor cores (4 is the workload's), and CUDA-core shapes."""
     spec = S.DecodeSpec("dec", B=2, Hq=Hq, Hkv=Hkv, L=2048, d=d, block_kv=bkv, tau=1e-2,
                         phi=1e-3, patience=2)
     _check_decode(spec, 1012, spec.tau, spec.phi, spec.patience)
