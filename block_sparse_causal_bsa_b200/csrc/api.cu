@@ -549,7 +549,7 @@ int bsa_score_path(const bsa_shape* s, bsa_score_kind kind) {
 
 int bsa_decode_path(const bsa_decode_shape* s) {
   if (!s || s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->L < 1 || s->Hq % s->Hkv) return -1;
-  return bsa::decode_tc_supported(*s) ? BSA_PATH_TENSOR_CORES : BSA_PATH_CUDA_CORES;
+  return bsa::decode_mma_supported(*s) ? BSA_PATH_TENSOR_CORES : BSA_PATH_CUDA_CORES;
 }
 
 }  // extern "C"

@@ -1,5 +1,5 @@
 // Decode attention with run-time termination ([ART] 2.1-2.4), CUDA-core kernel:
-// serves the shapes the tensor-core decode (decode_tc.cu) does not take
+// serves the shapes the tensor-core decode (decode_mma.cu) does not take
 // (d = 64, KV blocks of 64).
 //
 // One CTA per (batch, KV head). The CTA streams the KV cache in blocks of
@@ -281,8 +281,8 @@ cudaError_t launch_decode(const bsa_decode_shape& s, const bsa_decode_params& p,
   a.blist = block_list;
   a.bcnt = list_cnt;
   a.list_w = block_list ? list_w : 0;
-  if (decode_tc_supported(s))
-    return launch_decode_tc(s, a, q, kc, vc, out, blocks_used, probe_trace, dev_status, st);
+  if (decode_mma_supported(s))
+    return launch_decode_mma(s, a, q, kc, vc, out, blocks_used, probe_trace, dev_status, st);
   const int G = s.Hq / s.Hkv;
 #define BSA_DEC(D)                                                                             \
   switch (G) {                                                                                 \

@@ -103,11 +103,12 @@ struct DecodeArgs {
   int list_w;
 };
 
-// Decode with run-time termination on tcgen05 (bf16, d 128, KV blocks of 128, Hq/Hkv <= 8).
-bool decode_tc_supported(const bsa_decode_shape& s);
-cudaError_t launch_decode_tc(const bsa_decode_shape& s, const DecodeArgs& a, const void* q,
-                             const void* kc, const void* vc, void* out, int32_t* blocks_used,
-                             float* probe_trace, int32_t* dev_status, cudaStream_t st);
+// Decode with run-time termination on warp-level tensor-core MMAs (mma.sync; bf16, d 128,
+// KV blocks of 128, Hq/Hkv in {1, 2, 4, 8}).
+bool decode_mma_supported(const bsa_decode_shape& s);
+cudaError_t launch_decode_mma(const bsa_decode_shape& s, const DecodeArgs& a, const void* q,
+                              const void* kc, const void* vc, void* out, int32_t* blocks_used,
+                              float* probe_trace, int32_t* dev_status, cudaStream_t st);
 
 // Decode with run-time termination (dispatches to the tensor-core kernel where it applies).
 cudaError_t launch_decode(const bsa_decode_shape& s, const bsa_decode_params& p, const void* q,
