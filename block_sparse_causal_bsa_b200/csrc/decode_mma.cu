@@ -98,6 +98,12 @@ __device__ __forceinline__ void ldsm4_t(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
 }
+// sum over a warp of fp32 values, every lane returning the same value
+__device__ __forceinline__ float warp_sum_f32(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
 // transpose of an 8x8 b16 matrix held one row fragment per thread
 __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
   uint32_t y;
@@ -402,12 +408,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
     // the trace, and the fp64 products x_t^2 and x_t x_{t-1} (exact: products of fp32
     // values). The sums run across the warp in the fixed pairwise order of
     // warp_pairwise_sum; every lane then holds them and takes the same decision.
-    // ||x_{t-1}|| is the previous block's root (the same sum of the same values).
     const int np = a.n_probe;
     const int d0 = lane < np ? a.dims[lane] : 0;
     const int d1 = lane + 32 < np ? a.dims[lane + 32] : 0;
     float xp0 = 0.f, xp1 = 0.f;
-    double np_prev = 0.0;          // ||x_{t-1}||
+    float sp32 = 0.f, np32 = 0.f;  // the fp32 squared norm and norm of x_{t-1}
     int run = 0;
     for (int t = 0; t < ns; ++t) {
       const int slot = t & 1;
@@ -428,27 +433,63 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
         if (lane < np) tr[lane] = x0;
         if (lane + 32 < np) tr[lane + 32] = x1;
       }
-      const double sc2 = warp_pairwise_sum(
-          __dadd_rn(__dmul_rn((double)x0, (double)x0), __dmul_rn((double)x1, (double)x1)));
-      const double dt = warp_pairwise_sum(
-          __dadd_rn(__dmul_rn((double)x0, (double)xp0), __dmul_rn((double)x1, (double)xp1)));
-      xp0 = x0;
-      xp1 = x1;
-      const double nc = __dsqrt_rn(sc2);
+      // The test in fp32 first, then, only where that cannot decide, in fp64 as defined.
+      // With u = 2^-24, at most 64 coordinates (each term of a sum passes at most seven
+      // roundings) and both squared norms in [2^-60, 2^60], the fp32 values lie within
+      //   |ds32 - ds64| <= 5u (||x|| + ||x'||) + u ds32     (each norm to 4.6u)
+      //   |dd32 - dd64| <= 21u    (dot product to 7u ||x|| ||x'||, denominator to 10.2u,
+      //                            the divide and the subtract; |dot| <= ||x|| ||x'||)
+      // of the fp64 evaluation (whose own error is below 21 * 2^-53). The margins used
+      // below, 8u (||x|| + ||x'|| + ds32) and 32u, exceed these bounds with room for the
+      // rounding of the comparisons themselves, so a value outside them decides as the
+      // fp64 test would.
+      const float s32 = warp_sum_f32(__fadd_rn(__fmul_rn(x0, x0), __fmul_rn(x1, x1)));
+      const float d32 = warp_sum_f32(__fadd_rn(__fmul_rn(x0, xp0), __fmul_rn(x1, xp1)));
+      const float n32 = __fsqrt_rn(s32);
       bool stop = false;
       if (t >= 1) {
-        const double ds = fabs(__dadd_rn(nc, -np_prev));
-        bool stable = ds < (double)a.tau;
-        if (stable) {
-          // the direction term only matters once the norm term holds
-          const double den = __dmul_rn(nc, np_prev);
-          const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
-          stable = dd < (double)a.phi;
+        constexpr float kU = 0x1p-24f;
+        int verdict = -1;                                   // 0 / 1 decided, -1 open
+        if (!(a.tau > 0.f)) {
+          verdict = 0;                                      // ds >= 0 is never below it
+        } else if (s32 >= 0x1p-60f && s32 <= 0x1p60f && sp32 >= 0x1p-60f && sp32 <= 0x1p60f && isfinite(d32)) {
+          const float ds32 = fabsf(__fsub_rn(n32, np32));
+          const float e1 = 8.f * kU * (n32 + np32 + ds32);
+          if (ds32 - e1 >= a.tau) {
+            verdict = 0;
+          } else if (ds32 + e1 < a.tau) {
+            const float dd32 = __fsub_rn(1.f, __fdiv_rn(d32, __fmul_rn(n32, np32)));
+            const float e2 = 32.f * kU;
+            if (dd32 + e2 < a.phi) verdict = 1;
+            else if (dd32 - e2 >= a.phi) verdict = 0;
+          }
         }
-        run = stable ? run + 1 : 0;
+        if (verdict < 0) {
+          // the defining fp64 evaluation: exact products, pairwise sums, rounded root,
+          // product, divide and subtract
+          const double sc2 = warp_pairwise_sum(
+              __dadd_rn(__dmul_rn((double)x0, (double)x0), __dmul_rn((double)x1, (double)x1)));
+          const double sp2 = warp_pairwise_sum(
+              __dadd_rn(__dmul_rn((double)xp0, (double)xp0), __dmul_rn((double)xp1, (double)xp1)));
+          const double dt = warp_pairwise_sum(
+              __dadd_rn(__dmul_rn((double)x0, (double)xp0), __dmul_rn((double)x1, (double)xp1)));
+          const double nc = __dsqrt_rn(sc2), npv = __dsqrt_rn(sp2);
+          const double ds = fabs(__dadd_rn(nc, -npv));
+          bool stable = ds < (double)a.tau;
+          if (stable) {
+            const double den = __dmul_rn(nc, npv);
+            const double dd = (den == 0.0) ? 1.0 : __dadd_rn(1.0, -__ddiv_rn(dt, den));
+            stable = dd < (double)a.phi;
+          }
+          verdict = stable ? 1 : 0;
+        }
+        run = verdict ? run + 1 : 0;
         stop = a.enable && run >= a.patience;
       }
-      np_prev = nc;
+      xp0 = x0;
+      xp1 = x1;
+      sp32 = s32;
+      np32 = n32;
       if (lane == 0) {
         if (stop) {
           c.stop_at = t;

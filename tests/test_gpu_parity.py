@@ -199,6 +199,28 @@ def test_decode_limits():
     assert (used == 32).all()
 
 
+def test_decode_decider_at_its_thresholds():
+    """tau, then phi, set to the value the stability test computes on some block (its
+    minimum or median over the blocks of one group), so that a fast approximate screen of the
+    test cannot decide there and the defining fp64 evaluation has to: the stop must still
+    be the one the oracle's decision function gives on the GPU's probe trace."""
+    spec = S.DECODE_WORKLOADS["decode_art_64k"].scaled(B=1, L=4096)
+    (_, _, _), (qd, kd, vd) = _decode_inputs(spec, 1012)
+    dims = S.default_probe_dims(32)
+    _, _, trace, st = bb.decode(qd, kd, vd, block_kv=spec.block_kv, tau=0.0, phi=0.0, patience=1,
+                                enable=False, probe_dims=dims, want_trace=True)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    tr = trace.cpu().numpy()[0, 0]                      # group (0, 0), every block
+    steps = [O.probe_step(tr[t - 1], tr[t]) for t in range(1, tr.shape[0])]
+    ds = np.array([x[0] for x in steps])
+    dd = np.array([x[1] for x in steps])
+    f32 = lambda x: float(np.float32(x))
+    for tau, phi in ((f32(ds.min()), 2.0), (f32(np.sort(ds)[len(ds) // 2]), 2.0),
+                     (float("inf"), f32(dd.min())), (float("inf"), f32(np.sort(dd)[len(dd) // 2]))):
+        _check_decode(spec, 1012, tau, phi, 1)
+
+
 @pytest.mark.parametrize("nb", [1, 2, 3, 4, 5, 7, 9])
 def test_decode_stop_on_each_late_block(nb):
     """A stop on every block of short caches, the last two included: the kernel reads the
