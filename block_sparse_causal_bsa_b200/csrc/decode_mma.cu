@@ -10,9 +10,10 @@
 // single-CTA tcgen05.mma has a floor of ~80-130 cycles per instruction whatever
 // N is, and a 128-key block needs 16 of them in a dependent chain (~1900 cycles),
 // which set the period of the longest group's chain. An m16n8k16 mma.sync has a
-// ~20-cycle latency and four warps issue one every ~2 cycles per SM, so a block
-// costs a few hundred cycles and the chain becomes bound by the SM's own load
-// bandwidth (~180-240 GB/s for one SM streaming alone).
+// ~20-cycle latency and four warps issue one every ~2 cycles per SM, so the MMAs of
+// a block cost a few hundred cycles; what bounds the chain then is the block's
+// shared-memory traffic (64 KB of ldmatrix reads and the 64 KB TMA write) and the
+// SM's own load bandwidth (~180-240 GB/s for one SM streaming alone).
 //
 // One CTA per (batch, KV head), 192 threads:
 //   warp 0 (one thread)  TMA producer: K and V blocks of 128 keys (128-byte
@@ -29,9 +30,10 @@
 //   warp 5               decider: merges the four warps' states of block t into
 //                        x^(t) = O^(t)[first head][probe dims] / l (each warp's part
 //                        scaled by 2^(m_w - max m), added in warp order), then runs
-//                        the fp64 stability test (exact products, sums in a fixed
-//                        pairwise order across the warp) and publishes stop /
-//                        continue.
+//                        the stability test: in fp32 where proven margins to the
+//                        defining fp64 evaluation settle it, else in fp64 (exact
+//                        products, sums in a fixed pairwise order across the warp),
+//                        and publishes stop / continue.
 // The compute warps read the verdict on block t two blocks later, keeping their
 // state as of block t-2 until then; on a stop they return that copy. After a stop
 // the producer is released through a halt flag; a compute warp that waits for a
@@ -404,10 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(
   } else if (warp == 5) {
     // ---------------- decider ----------------
     // Lane i owns probe coordinates i and i + 32: it merges the four warps' parts of the
-    // first head for them, forms x = O / l (the fp32 divisions run in parallel), writes
-    // the trace, and the fp64 products x_t^2 and x_t x_{t-1} (exact: products of fp32
-    // values). The sums run across the warp in the fixed pairwise order of
-    // warp_pairwise_sum; every lane then holds them and takes the same decision.
+    // first head for them, forms x = O / l (the fp32 divisions run in parallel) and writes
+    // the trace. The sums of the test run across the warp (every lane then holds them and
+    // takes the same decision); in the fp64 evaluation the products are exact (products
+    // of fp32 values) and the sums take the fixed pairwise order of warp_pairwise_sum.
     const int np = a.n_probe;
     const int d0 = lane < np ? a.dims[lane] : 0;
     const int d1 = lane + 32 < np ? a.dims[lane + 32] : 0;
