@@ -2,8 +2,9 @@
 run-time termination.
 
 One step = one pass of the prefill hot path over one batch: pool + block score
-(bsa_score) -> top-k with uncertainty gate (bsa_select) -> block-sparse attend
-(bsa_attend), on the gated 128k workload (B=1, 32 query / 8 KV heads,
+with the per-row top-k ranked inside the score kernel, uncertainty gate and
+kv_idx (bsa_score_select) -> block-sparse attend (bsa_attend), on the gated 128k
+workload (B=1, 32 query / 8 KV heads,
 N=131072, d=128, key block 64, query tile 128, k=64, rho=2, quantile 0.25).
 value = effective TFLOP/s = (4 * tile_q * block_k * d per selected block, from
 kv_cnt) / device time of the whole step. The decode row (batch 16, 64k cache,
