@@ -548,7 +548,13 @@ int bsa_score_path(const bsa_shape* s, bsa_score_kind kind) {
 }
 
 int bsa_decode_path(const bsa_decode_shape* s) {
+  // the shape checks of bsa_decode (check_decode), without the pointers and parameters
   if (!s || s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->L < 1 || s->Hq % s->Hkv) return -1;
+  const int G = s->Hq / s->Hkv;
+  if ((G != 1 && G != 2 && G != 4 && G != 8) || (s->d != 64 && s->d != 128) ||
+      (s->block_kv != 64 && s->block_kv != 128) || s->L % s->block_kv ||
+      (long long)s->B * s->Hkv * s->L >= (1ll << 31) || s->dtype != BSA_BF16)
+    return -1;
   return bsa::decode_mma_supported(*s) ? BSA_PATH_TENSOR_CORES : BSA_PATH_CUDA_CORES;
 }
 

@@ -368,9 +368,9 @@ bsa_status bsa_selftest_wait(int mode, int32_t* dev_status, int32_t* completed, 
  *   bsa_attend_path  tensor cores for bf16, d = 128, key blocks of 64, query tiles of 128,
  *                    W <= 1024 and B*Hq*N < 2^31; CUDA cores for every other shape
  *                    (BSA_F32, d = 64, key blocks of 128, query tiles of 64, W > 1024).
- *   bsa_decode_path  tensor cores for bf16, d = 128, block_kv = 128, Hq/Hkv in
- *                    {1, 2, 4, 8} and B*Hkv*L < 2^31; CUDA cores for every other shape
- *                    (BSA_F32, d = 64, block_kv = 64).
+ *   bsa_decode_path  tensor cores for d = 128 and block_kv = 128; CUDA cores for d = 64
+ *                    or block_kv = 64 (decode takes bf16 caches, Hq/Hkv in {1, 2, 4, 8}
+ *                    and B*Hkv*L < 2^31 only; -1 otherwise).
  * bsa_attend_vs always runs on tensor cores (other shapes are rejected). */
 enum { BSA_PATH_CUDA_CORES = 0, BSA_PATH_TENSOR_CORES = 1 };
 int bsa_score_path(const bsa_shape* shape, bsa_score_kind kind);

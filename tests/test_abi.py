@@ -287,4 +287,10 @@ def test_kernel_path_queries():
     assert bb.bsa_decode_path(bb.DecodeShape(2, 8, 8, 4096, 128, 128, bb.BSA_BF16)) == TC
     assert bb.bsa_decode_path(bb.DecodeShape(2, 8, 2, 4096, 64, 128, bb.BSA_BF16)) == CC
     assert bb.bsa_decode_path(bb.DecodeShape(2, 8, 2, 4096, 128, 64, bb.BSA_BF16)) == CC
+    for hq, hkv in ((2, 2), (4, 2), (8, 1)):           # group sizes 1, 2, 8
+        assert bb.bsa_decode_path(bb.DecodeShape(2, hq, hkv, 4096, 128, 128, bb.BSA_BF16)) == TC
+    # shapes bsa_decode itself rejects: fp32 caches, a group of 3, L not a block multiple
+    assert bb.bsa_decode_path(bb.DecodeShape(2, 8, 2, 4096, 128, 128, bb.BSA_F32)) == -1
+    assert bb.bsa_decode_path(bb.DecodeShape(2, 6, 2, 4096, 128, 128, bb.BSA_BF16)) == -1
+    assert bb.bsa_decode_path(bb.DecodeShape(2, 8, 2, 4000, 128, 128, bb.BSA_BF16)) == -1
     assert bb.bsa_decode_path(bb.DecodeShape(2, 6, 4, 4096, 128, 128, bb.BSA_BF16)) == -1
